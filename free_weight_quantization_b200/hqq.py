@@ -1,0 +1,163 @@
+"""Python binding of the C ABI in include/hqq_b200.h (argument marshalling only).
+
+Every step of quantize and dequantize runs in the CUDA kernels of libhqq_b200.so; this module
+allocates output buffers with torch when the caller does not pass them, hands raw device
+pointers and the current CUDA stream to the library, and raises on a non-zero return code.
+There is no CPU fallback: loading fails loudly when the library is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libhqq_b200.so")
+
+HQQ_OK = 0
+HQQ_MAX_GROUP_SIZE = 256
+HQQ_MAX_ITERS = 64
+
+
+class HqqOpt(ctypes.Structure):
+    _fields_ = [("iters", ctypes.c_int32), ("lp_norm", ctypes.c_double),
+                ("beta", ctypes.c_double), ("kappa", ctypes.c_double),
+                ("eps_tiny", ctypes.c_float), ("scale_max", ctypes.c_float)]
+
+
+class HqqError(RuntimeError):
+    pass
+
+
+_lib = None
+
+# (name, restype, argtypes) of every symbol the header declares
+_P, _I64, _I32, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+SIGNATURES = {
+    "hqq_default_opt": (None, [ctypes.POINTER(HqqOpt)]),
+    "hqq_packed_bytes": (_I64, [_I64, _I32]),
+    "hqq_quantize_workspace_bytes": (_SZ, [_I64, _I64, _I32, _I64, _I32, _I32]),
+    "hqq_quantize": (_I32, [_P, _I64, _I64, _I32, _I64, _I32, ctypes.POINTER(HqqOpt), _P, _P, _P,
+                            _P, _P, _P, _P, _P, _SZ, _P]),
+    "hqq_dequantize": (_I32, [_P, _P, _P, _I64, _I64, _I32, _I64, _I32, _P, _P]),
+    "hqq_strerror": (ctypes.c_char_p, [_I32]),
+}
+
+
+def lib():
+    """The loaded CUDA library; raises if libhqq_b200.so has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise HqqError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m free_weight_quantization_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(rc: int, what: str):
+    if rc != HQQ_OK:
+        raise HqqError(f"{what}: {lib().hqq_strerror(rc).decode()} (code {rc})")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def default_opt() -> HqqOpt:
+    o = HqqOpt()
+    lib().hqq_default_opt(ctypes.byref(o))
+    return o
+
+
+def hqq_packed_bytes(n: int, nbits: int) -> int:
+    return int(lib().hqq_packed_bytes(n, nbits))
+
+
+def hqq_quantize_workspace_bytes(rows: int, cols: int, nbits: int, group_size: int, axis: int,
+                                 iters: int) -> int:
+    return int(lib().hqq_quantize_workspace_bytes(rows, cols, nbits, group_size, axis, iters))
+
+
+@dataclass
+class Quantized:
+    """Packed codes + fp16 metadata (the page's W_q, scale = Delta = 1/s, zero) and the shape."""
+    packed: torch.Tensor
+    scale: torch.Tensor
+    zero: torch.Tensor
+    rows: int
+    cols: int
+    nbits: int
+    group_size: int
+    axis: int
+    iters_run: torch.Tensor | None = None
+    s: torch.Tensor | None = None
+    z: torch.Tensor | None = None
+    err_trace: torch.Tensor | None = None
+
+
+def hqq_quantize(W: torch.Tensor, nbits: int = 4, group_size: int = 64, axis: int = 1,
+                 iters: int = 20, lp_norm: float = 0.7, beta: float = 10.0, kappa: float = 1.01,
+                 eps_tiny: float = 1e-4, scale_max: float = 2e4, *, out: Quantized | None = None,
+                 workspace: torch.Tensor | None = None, debug: bool = False,
+                 stream: torch.cuda.Stream | None = None) -> Quantized:
+    """HQQ quantize + pack of an fp16 CUDA matrix [rows, cols] (see hqq_quantize in the header).
+    With debug=True also returns iters_run, binary32 s and z, and the exact error trace."""
+    if W.dtype != torch.float16 or not W.is_cuda or W.dim() != 2 or not W.is_contiguous():
+        raise HqqError("W must be a contiguous 2-D float16 CUDA tensor")
+    rows, cols = W.shape
+    N = rows * cols
+    if group_size <= 0 or N % group_size:
+        raise HqqError("rows*cols must be a positive multiple of group_size")
+    G = N // group_size
+    dev = W.device
+    if out is None:
+        pb = hqq_packed_bytes(N, nbits)
+        if pb < 0:
+            raise HqqError("nbits must be 2, 3 or 4")
+        out = Quantized(torch.empty(max(pb, 1), dtype=torch.uint8, device=dev),
+                        torch.empty(G, dtype=torch.float16, device=dev),
+                        torch.empty(G, dtype=torch.float16, device=dev),
+                        rows, cols, nbits, group_size, axis)
+        if debug:
+            out.iters_run = torch.zeros(1, dtype=torch.int32, device=dev)
+            out.s = torch.empty(G, dtype=torch.float32, device=dev)
+            out.z = torch.empty(G, dtype=torch.float32, device=dev)
+            out.err_trace = torch.zeros(max(2 * iters, 2), dtype=torch.int64, device=dev)
+    wsb = hqq_quantize_workspace_bytes(rows, cols, nbits, group_size, axis, iters)
+    if workspace is None:
+        workspace = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+    opt = HqqOpt(iters, lp_norm, beta, kappa, eps_tiny, scale_max)
+    st = stream if stream is not None else torch.cuda.current_stream(dev)
+    rc = lib().hqq_quantize(_ptr(W), rows, cols, nbits, group_size, axis, ctypes.byref(opt),
+                            _ptr(out.packed), _ptr(out.scale), _ptr(out.zero), _ptr(out.iters_run),
+                            _ptr(out.s), _ptr(out.z), _ptr(out.err_trace), _ptr(workspace),
+                            workspace.numel() * workspace.element_size(),
+                            ctypes.c_void_p(st.cuda_stream))
+    _check(rc, "hqq_quantize")
+    return out
+
+
+def hqq_dequantize(q: Quantized, out: torch.Tensor | None = None,
+                   stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """Unpack + (q - zero) * scale -> fp16 [rows, cols] (see hqq_dequantize in the header)."""
+    if out is None:
+        out = torch.empty(q.rows, q.cols, dtype=torch.float16, device=q.packed.device)
+    st = stream if stream is not None else torch.cuda.current_stream(q.packed.device)
+    rc = lib().hqq_dequantize(_ptr(q.packed), _ptr(q.scale), _ptr(q.zero), q.rows, q.cols, q.nbits,
+                              q.group_size, q.axis, _ptr(out), ctypes.c_void_p(st.cuda_stream))
+    _check(rc, "hqq_dequantize")
+    return out
+
+
+def err_trace_ints(t: torch.Tensor, n: int) -> list[int]:
+    """Exact per-round error sums (units of 2^-32) from the (low, high) uint64 pairs."""
+    v = t.cpu().view(torch.int64).tolist()
+    return [(v[2 * i] & (2 ** 64 - 1)) + ((v[2 * i + 1] & (2 ** 64 - 1)) << 64) for i in range(n)]

@@ -1,0 +1,131 @@
+/*
+ * hqq_b200.h -- C ABI of the B200 (sm_100a) HQQ group-wise weight quantizer.
+ *
+ * The method is the one described on the page "HQQ 算法解读：不用校准数据，怎样把大模型权重压到
+ * 4 bit" (ludovicoyin.github.io/blog/posts/hqq-half-quadratic-quantization), cited as
+ * [HQQ 算法解读, <section>].  Its Python interface there is BaseQuantizeConfig(nbits,
+ * group_size, axis) plus HQQLinear(...) and .dequantize() (section "一个最小可复现实验"); this
+ * header restates quantize and dequantize as two calls on caller-owned device buffers.
+ *
+ * Conventions for every call below:
+ *   - all data pointers are DEVICE pointers owned by the caller; the library allocates
+ *     nothing and keeps no pointer after the call returns;
+ *   - calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default stream);
+ *     the return value reports argument checks and launch errors only;
+ *   - W is fp16, row-major [rows, cols], never modified; N = rows * cols, G = N / group_size;
+ *   - group view [HQQ 算法解读, "`axis` 不是一个无关紧要的开关"]: axis = 1 takes groups of
+ *     group_size consecutive elements (W.reshape([-1, g])); axis = 0 takes the columns of
+ *     the [g, G] row-major view (W.reshape([g, -1])), i.e. group k = elements j*G + k;
+ *   - packed codes are in flat row-major element order for both axes, lowest index in the
+ *     lowest bits [HQQ 算法解读, "为什么一定要分组"]: 4 bit = two codes per byte, 2 bit = four
+ *     codes per byte, 3 bit = ten codes per little-endian 32-bit word (bits 30-31 zero); the
+ *     tail of the last byte or word is zero;
+ *   - metadata [HQQ 算法解读, "量化公式：把尺子写出来"]: scale[G] = fp16(1/s) (the page's
+ *     Delta) and zero[G] = fp16(z), in group order.
+ *   - W must hold finite values.
+ */
+#ifndef HQQ_B200_H
+#define HQQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* return codes */
+#define HQQ_OK 0
+#define HQQ_ERR_ARG 1          /* a size, bit width, axis, option or required pointer is invalid */
+#define HQQ_ERR_ALIGN 2        /* a pointer is not aligned as documented */
+#define HQQ_ERR_WORKSPACE 3    /* workspace null or smaller than hqq_quantize_workspace_bytes() */
+#define HQQ_ERR_CUDA 4         /* a CUDA runtime call or kernel launch failed */
+#define HQQ_ERR_UNSUPPORTED 5  /* valid for the method, outside this library's limits (below) */
+
+/* limits of this library */
+#define HQQ_MAX_GROUP_SIZE 256 /* group_size 1 .. 256 */
+#define HQQ_MAX_ITERS 64       /* iters 0 .. 64 (the page's default is 20) */
+
+/*
+ * Options of the proximal loop [HQQ 算法解读, "第一拍" and "第二拍"].
+ *   iters      at most this many rounds (page: 20)
+ *   lp_norm    p of the lp shrink, 0 < p < 2 (page: 0.7)
+ *   beta       beta of the first round, > 0 (page: 10)
+ *   kappa      beta is multiplied by kappa after each round, > 0 (page: 1.01)
+ *   eps_tiny   a group whose max - min is below this gets s = 1 (the page only says "too
+ *              small"; 1e-4 is this library's reading), >= 0
+ *   scale_max  s is clamped to at most this value (page: 2e4), > 0
+ */
+typedef struct hqq_opt {
+    int32_t iters;
+    double lp_norm;
+    double beta;
+    double kappa;
+    float eps_tiny;
+    float scale_max;
+} hqq_opt_t;
+
+/* Fills *opt with the page's defaults: 20, 0.7, 10, 1.01, 1e-4, 2e4. */
+void hqq_default_opt(hqq_opt_t *opt);
+
+/* Exact size in bytes of the packed codes of n weights: n/2, n/4 or 4*ceil(n/10), rounded up
+ * [HQQ 算法解读, "为什么一定要分组"].  Returns -1 for nbits outside {2, 3, 4} or n < 0. */
+int64_t hqq_packed_bytes(int64_t n, int nbits);
+
+/* Device workspace, in bytes, that hqq_quantize needs for these arguments (0 if invalid). */
+size_t hqq_quantize_workspace_bytes(int64_t rows, int64_t cols, int nbits, int64_t group_size,
+                                    int axis, int iters);
+
+/*
+ * HQQ quantize + pack [HQQ 算法解读, "第一拍", "第二拍", "为什么一定要分组"]:
+ * per group s0 = (2^b-1)/(max-min) (s = 1 when max-min < eps_tiny, then s <= scale_max),
+ * z0 = -min*s0; then up to `iters` rounds of q = clip(round(W*s+z), 0, 2^b-1),
+ * W_hat = (q-z)/s, e = shrink_lp(W - W_hat, beta_i), z <- mean(q - (W-e)*s), with
+ * beta_i = beta*kappa^i; the loop stops at the first round whose tensor-wide MAE
+ * mean|W - W_hat| is not strictly below the best so far and keeps the zero of the best
+ * round; a final quantize with the original W gives the codes.
+ *
+ * Arguments
+ *   W            [rows*cols] fp16, 16-byte aligned
+ *   nbits        2, 3 or 4;  group_size 1..256 dividing rows*cols;  axis 0 or 1
+ *   opt          options (host pointer); NULL = hqq_default_opt()
+ *   packed       [hqq_packed_bytes(N, nbits)] bytes, 16-byte aligned (output)
+ *   scale, zero  [G] fp16 each, 2-byte aligned (outputs): fp16(1/s) and fp16(z)
+ *   iters_run    device int32, nullable (output): rounds whose MAE was computed
+ *   s_f32, z_f32 [G] float each, nullable (outputs): s and the kept z in binary32
+ *   err_trace    [2*iters] uint64, nullable (output): entry i < iters_run is the exact sum
+ *                over groups of floor(2^32 * sum_group |W - W_hat|) at round i, as
+ *                (low 64 bits, high 64 bits); MAE_i = that / 2^32 / N.  Entries at or past
+ *                iters_run are unspecified.
+ *   workspace    >= hqq_quantize_workspace_bytes(...) bytes, 16-byte aligned; contents on
+ *                entry do not matter; must not be used by anything else until the work
+ *                queued on `stream` by this call has finished
+ *   stream       cudaStream_t
+ * Returns HQQ_OK or an HQQ_ERR_* code; on an error nothing is launched.
+ */
+int hqq_quantize(const void *W, int64_t rows, int64_t cols, int nbits, int64_t group_size,
+                 int axis, const hqq_opt_t *opt, void *packed, void *scale, void *zero,
+                 int32_t *iters_run, float *s_f32, float *z_f32, uint64_t *err_trace,
+                 void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Unpack + dequantize [HQQ 算法解读, "量化公式" and "从压缩文件到一次前向"]:
+ * W_out = fp16((q - f32(zero)) * f32(scale)) in binary32, rounded once to fp16, written in
+ * the original [rows, cols] row-major layout.
+ *   packed   as written by hqq_quantize, 16-byte aligned
+ *   scale, zero [G] fp16, 2-byte aligned
+ *   W_out    [rows*cols] fp16, 16-byte aligned (output)
+ * Returns HQQ_OK or an HQQ_ERR_* code; on an error nothing is launched.
+ */
+int hqq_dequantize(const void *packed, const void *scale, const void *zero, int64_t rows,
+                   int64_t cols, int nbits, int64_t group_size, int axis, void *W_out,
+                   void *stream);
+
+/* Text for a return code (static storage). */
+const char *hqq_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HQQ_B200_H */

@@ -1,0 +1,118 @@
+"""The C-ABI library: it loads, exports every symbol the header declares, and rejects bad
+arguments on the host before anything reaches a GPU (these tests run without one)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from free_weight_quantization_b200 import build as fbuild
+from free_weight_quantization_b200 import hqq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hqq_b200.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    fbuild.build()
+    return hqq.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(hqq_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_symbols_exported(L):
+    names = declared_functions()
+    assert {"hqq_quantize", "hqq_dequantize", "hqq_packed_bytes",
+            "hqq_quantize_workspace_bytes", "hqq_default_opt", "hqq_strerror"} <= set(names)
+    raw = ctypes.CDLL(hqq.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), n
+    assert set(names) == set(hqq.SIGNATURES), "binding and header disagree"
+
+
+def test_default_opt_is_the_pages_defaults(L):
+    o = hqq.default_opt()
+    assert (o.iters, o.lp_norm, o.beta, o.kappa) == (20, 0.7, 10.0, 1.01)
+    assert abs(o.eps_tiny - 1e-4) < 1e-9 and o.scale_max == 2e4
+
+
+@pytest.mark.parametrize("nbits", [2, 3, 4])
+@pytest.mark.parametrize("n", [0, 1, 7, 10, 64, 4096 * 4096, 4096 * 11008 + 3])
+def test_packed_bytes_match_oracle(L, nbits, n):
+    assert hqq.hqq_packed_bytes(n, nbits) == oracle.packed_bytes(n, nbits)
+
+
+def test_packed_bytes_rejects(L):
+    assert hqq.hqq_packed_bytes(10, 5) == -1
+    assert hqq.hqq_packed_bytes(-1, 4) == -1
+
+
+def test_workspace_bytes(L):
+    ws = hqq.hqq_quantize_workspace_bytes
+    assert ws(4096, 4096, 4, 64, 1, 20) > 0
+    assert ws(4096, 4096, 4, 64, 1, 20) < 4096 * 4096 // 16  # small: round sums + 1 byte/group
+    assert ws(10, 10, 4, 3, 1, 20) == 0        # 100 % 3 != 0
+    assert ws(16, 16, 5, 16, 1, 20) == 0       # 5 bits
+    assert ws(16, 16, 4, 16, 2, 20) == 0       # axis 2
+    assert ws(16, 1024, 4, 512, 1, 20) == 0    # group beyond the library limit
+    assert ws(16, 16, 4, 16, 1, 65) == 0       # iters beyond the library limit
+    # axis=0 whose packed words do not line up with tiles needs byte staging of all codes
+    assert ws(8, 6, 4, 2, 0, 20) >= 48
+
+
+FAKE = 0x10000  # never dereferenced: every call below fails its host-side checks first
+
+
+def q(L, W=FAKE, rows=64, cols=64, nbits=4, g=64, axis=1, opt=None, packed=FAKE, scale=FAKE,
+      zero=FAKE, ws=FAKE, wsb=1 << 20, iters_run=None):
+    P = ctypes.c_void_p
+    return L.hqq_quantize(P(W), rows, cols, nbits, g, axis, opt, P(packed), P(scale), P(zero),
+                          P(iters_run) if iters_run else None, None, None, None, P(ws), wsb, None)
+
+
+def test_quantize_rejects_on_host(L):
+    assert q(L, nbits=5) == 1
+    assert q(L, nbits=1) == 1
+    assert q(L, axis=3) == 1
+    assert q(L, g=0) == 1
+    assert q(L, rows=0) == 1
+    assert q(L, cols=-4) == 1
+    assert q(L, g=48) == 1                     # 4096 % 48 != 0
+    assert q(L, rows=2, cols=512, g=512) == 5  # group_size > 256
+    assert q(L, W=0) == 1
+    assert q(L, packed=0) == 1
+    assert q(L, W=FAKE + 2) == 2               # W not 16-byte aligned
+    assert q(L, packed=FAKE + 4) == 2
+    assert q(L, scale=FAKE + 1) == 2
+    assert q(L, iters_run=FAKE + 2) == 2
+    assert q(L, ws=0) == 3
+    assert q(L, wsb=16) == 3
+    assert q(L, ws=FAKE + 8) == 2
+    for field, bad in [("lp_norm", 0.0), ("lp_norm", 2.0), ("beta", 0.0), ("kappa", -1.0),
+                       ("scale_max", 0.0), ("eps_tiny", -1.0), ("iters", -1), ("iters", 65)]:
+        o = hqq.default_opt()
+        setattr(o, field, bad)
+        rc = q(L, opt=ctypes.byref(o))
+        assert rc == (5 if (field, bad) == ("iters", 65) else 1), (field, bad, rc)
+
+
+def test_dequantize_rejects_on_host(L):
+    P = ctypes.c_void_p
+    d = L.hqq_dequantize
+    assert d(P(FAKE), P(FAKE), P(FAKE), 64, 64, 5, 64, 1, P(FAKE), None) == 1
+    assert d(P(FAKE), P(FAKE), P(FAKE), 64, 64, 4, 63, 1, P(FAKE), None) == 1
+    assert d(None, P(FAKE), P(FAKE), 64, 64, 4, 64, 1, P(FAKE), None) == 1
+    assert d(P(FAKE + 4), P(FAKE), P(FAKE), 64, 64, 4, 64, 1, P(FAKE), None) == 2
+    assert d(P(FAKE), P(FAKE), P(FAKE), 64, 64, 4, 64, 1, P(FAKE + 2), None) == 2
+
+
+def test_strerror(L):
+    for code in range(6):
+        assert L.hqq_strerror(code)
+    assert L.hqq_strerror(99) == b"unknown error"

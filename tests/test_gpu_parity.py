@@ -1,0 +1,153 @@
+"""CUDA path vs the CPU oracle on the same seeded inputs (needs a B200)."""
+import concurrent.futures as cf
+import multiprocessing as mp
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import parity
+from free_weight_quantization_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def pool():
+    # spawn: a forked child of a process that has touched CUDA can hang
+    ex = cf.ProcessPoolExecutor(max_workers=min(4, os.cpu_count() or 1),
+                                mp_context=mp.get_context("spawn"))
+    yield ex
+    ex.shutdown(cancel_futures=True)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from free_weight_quantization_b200 import build
+    build.build()
+    assert torch.cuda.is_available(), "these tests need a CUDA device"
+
+
+def _bimodal(rows, cols, seed):
+    r = np.random.default_rng(seed)
+    return (np.where(r.random((rows, cols)) < 0.5, -1.0, 1.0)
+            * (1 + 0.01 * r.standard_normal((rows, cols)))).astype(np.float16)
+
+
+def _sparse(rows, cols, seed):
+    r = np.random.default_rng(seed)
+    return (r.standard_normal((rows, cols)) * (r.random((rows, cols)) < 0.1)).astype(np.float16)
+
+
+def _wide(rows, cols, seed):
+    return (np.random.default_rng(seed).standard_normal((rows, cols)) * 3.0).astype(np.float16)
+
+
+def _const(rows, cols, seed):
+    W = np.full((rows, cols), 0.375, np.float16)
+    W[rows // 2:] = -1.25
+    return W
+
+
+def _tiny_range(rows, cols, seed):
+    r = np.random.default_rng(seed)
+    W = 0.5 + r.integers(0, 3, (rows, cols)) * 2.0 ** -11     # ranges of 0 .. 1e-3
+    return W.astype(np.float16)
+
+
+GENS = {"t": wl.student_t, "n": wl.outlier_normal, "bimodal": _bimodal, "sparse": _sparse,
+        "wide": _wide, "const": _const, "tiny": _tiny_range}
+
+# rows, cols, nbits, group_size, axis, iters, generator
+EDGE = [
+    (1, 64, 4, 64, 1, 20, "t"),          # one group
+    (1, 64, 4, 64, 1, 20, "const"),
+    (4, 64, 4, 64, 1, 20, "tiny"),        # ranges around eps_tiny: s = 1 or clamped 2e4
+    (3, 160, 3, 16, 1, 20, "t"),
+    (7, 33, 4, 3, 1, 20, "t"),            # g = 3, odd N (last nibble), many tiles of 320 groups
+    (5, 50, 3, 25, 1, 7, "t"),
+    (9, 100, 2, 12, 1, 20, "t"),
+    (64, 96, 4, 48, 1, 20, "t"),          # group padded to 64 slots
+    (16, 4096, 4, 256, 1, 20, "t"),       # largest group
+    (64, 64, 4, 64, 1, 0, "t"),           # no rounds: min-max RTN
+    (64, 64, 4, 64, 1, 1, "t"),
+    (64, 128, 4, 64, 1, 64, "t"),         # most rounds
+    (64, 256, 4, 64, 1, 20, "wide"),      # lp shrink active
+    (64, 256, 2, 16, 1, 20, "wide"),
+    (64, 256, 3, 64, 1, 20, "wide"),
+    (64, 256, 4, 64, 1, 20, "bimodal"),   # early global stop: stale groups are recomputed
+    (64, 256, 2, 16, 1, 20, "bimodal"),
+    (64, 256, 3, 64, 1, 20, "bimodal"),
+    (64, 256, 4, 32, 1, 20, "sparse"),
+    (300, 512, 4, 64, 1, 20, "n"),        # 15 tiles
+    (333, 64, 3, 64, 1, 20, "t"),         # ragged last tile
+    (256, 128, 4, 128, 0, 20, "t"),       # axis 0, aligned
+    (128, 80, 3, 16, 0, 20, "t"),         # axis 0, G = 640
+    (32, 64, 2, 32, 0, 20, "t"),          # axis 0, G = 64
+    (30, 32, 4, 16, 0, 20, "t"),          # axis 0, G = 60: byte staging + pack kernel
+    (40, 41, 3, 8, 0, 20, "t"),           # axis 0, G = 205, odd
+    (64, 256, 4, 64, 0, 20, "bimodal"),
+    (64, 256, 4, 64, 0, 20, "wide"),
+]
+
+
+@pytest.mark.parametrize("case", EDGE, ids=lambda c: "x".join(map(str, c)))
+def test_edge_case(case):
+    rows, cols, nbits, g, axis, iters, gen = case
+    W = GENS[gen](rows, cols, 17 + rows)
+    ref = parity.oracle_on(W, nbits, g, axis, iters)
+    got = parity.gpu_quantize(W, nbits, g, axis, iters)
+    parity.check(W, ref, got, str(case))
+
+
+def test_small_config_and_repeat():
+    c = wl.SMALL
+    W = c.make()
+    ref = parity.oracle_on(W, c.nbits, c.group_size, c.axis)
+    a = parity.gpu_quantize(W, c.nbits, c.group_size, c.axis)
+    parity.check(W, ref, a, c.name)
+    b = parity.gpu_quantize(W, c.nbits, c.group_size, c.axis)  # repeat: deterministic
+    assert np.array_equal(a["packed"], b["packed"]) and np.array_equal(a["deq"], b["deq"])
+
+
+@pytest.mark.parametrize("case", wl.CASES[1:], ids=lambda c: c.name)
+def test_full_size_config(case, pool):
+    fut = pool.submit(parity.oracle_job, case.name)
+    W = case.make()
+    got = parity.gpu_quantize(W, case.nbits, case.group_size, case.axis)
+    ref = fut.result()
+    stats = parity.check(W, ref, got, case.name)
+    print(case.name, ref["iters_run"], stats)
+
+
+@pytest.mark.parametrize("nbits", [2, 3, 4])
+@pytest.mark.parametrize("shape,g,axis", [((64, 64), 64, 1), ((37, 129), 3, 1), ((100, 7), 10, 1),
+                                          ((256, 64), 128, 0), ((30, 32), 16, 0),
+                                          ((41, 40), 8, 0)])
+def test_dequant_random_codes(nbits, shape, g, axis):
+    from free_weight_quantization_b200 import hqq
+    rows, cols = shape
+    N = rows * cols
+    r = np.random.default_rng(N + nbits)
+    codes = r.integers(0, 1 << nbits, N).astype(np.uint8)
+    packed = oracle.pack(codes, nbits)
+    G = N // g
+    scale = (r.random(G) * 0.05 + 1e-3).astype(np.float16)
+    zero = (r.random(G) * (1 << nbits)).astype(np.float16)
+    ref = oracle.dequant(packed, scale, zero, rows, cols, nbits, g, axis)
+    buf = np.zeros((packed.size + 15) // 16 * 16, np.uint8)
+    buf[:packed.size] = packed
+    q = hqq.Quantized(torch.from_numpy(buf).cuda(), torch.from_numpy(scale).cuda(),
+                      torch.from_numpy(zero).cuda(), rows, cols, nbits, g, axis)
+    out = hqq.hqq_dequantize(q).cpu().numpy()
+    assert np.array_equal(out.view(np.uint16), ref.view(np.uint16))
+
+
+def test_native_library_is_loaded():
+    from free_weight_quantization_b200 import hqq
+    hqq.lib()
+    maps = open("/proc/self/maps").read()
+    assert "libhqq_b200.so" in maps

@@ -1,0 +1,331 @@
+"""Benchmark: HQQ quantize+pack and dequantize of a 4096x4096 fp16 weight on B200.
+
+One step = the whole hot path over one matrix: hqq_quantize (min-max init, proximal rounds
+with the tensor-wide stop rule, final quantize, bit-packing, fp16 metadata) followed by
+hqq_dequantize.  Inputs rotate over R copies so that every step reads its matrix from HBM
+(R * 33.5 MB > 126 MB of L2).  Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+--impl reference times the CPU oracle (the plain C reference of the method) on the host on a
+bounded slice of the same workload.  Under torchrun every rank quantizes its own matrices (no
+data-path communication: weak scaling); the reference arm runs on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "HQQ quantize+pack Gweights/s at 4096² 4-bit g64; dequant GB/s; % of HBM peak"
+UNIT = "Gweights/s"
+ROWS = COLS = 4096
+NBITS, GROUP, AXIS, ITERS = 4, 64, 1, 20
+WORKLOAD = ("0.02*StudentT(4) clipped to +-1, fp16 4096x4096 (attention-projection-shaped), seed 1; "
+            "4-bit, group 64, axis 1, <=20 rounds, p=0.7, beta=10, kappa=1.01")
+ROTATE = 8
+ISSUE_LANES_PER_SM = 128     # 4 SM sub-partitions x 32 lanes issue one instruction per clock
+ALU_OPS_INIT, ALU_OPS_ROUND, ALU_OPS_FINAL = 3, 12, 6   # algorithmic ops per weight
+
+
+def peaks():
+    p = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "src": "fallback"}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            m = json.load(f)
+        p.update(hbm_gbs=float(m["hbm_gbs"]), sm_max_mhz=float(m.get("sm_max_mhz", 1965.0)),
+                 src="measured")
+    except (OSError, KeyError, ValueError):
+        pass
+    return p
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms in the background."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            return self
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        win = [p for t, p in self.samples if t0 <= t <= t1]
+        window = "timed"
+        if len(win) < 3:
+            win = [p for _, p in self.samples]
+            window = "whole run"
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(p[1]) for p in win if num(p[1]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for p in win for n, v in zip(names, p[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": num(win[0][2]), "reasons": reasons, "samples": len(win),
+                "window": window, "power_w_max": max((num(p[3]) or 0.0) for p in win)}
+
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def run_reference(args, ws, rank):
+    """The CPU oracle, as it stands, on a bounded slice of the workload."""
+    if rank != 0:
+        return
+    import numpy as np
+
+    import oracle
+    from free_weight_quantization_b200 import workloads as wl
+    oracle.build()
+    W = wl.ATTN.make()
+    rows = 256                        # each step: a 256 x 4096 slice (1 M weights)
+    times = []
+    for i in range(args.warmup + args.steps):
+        sl = np.ascontiguousarray(W[(i % 16) * rows:(i % 16 + 1) * rows])
+        t0 = time.perf_counter()
+        r = oracle.quantize(sl, NBITS, GROUP, AXIS, iters=ITERS)
+        oracle.dequant(r["packed"], r["scale"], r["zero"], rows, COLS, NBITS, GROUP, AXIS)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    n = rows * COLS
+    value = n * len(times) / sum(times) / 1e9
+    sample = f"{args.steps} slices of 256x4096 rows of the 4096x4096 workload, quantize+pack+dequant"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample_rows": rows},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline():
+    """The oracle timed once on the full 4096x4096 matrix (about 15 s on one core)."""
+    import oracle
+    from free_weight_quantization_b200 import workloads as wl
+    oracle.build()
+    W = wl.ATTN.make()
+    t0 = time.perf_counter()
+    r = oracle.quantize(W, NBITS, GROUP, AXIS, iters=ITERS)
+    oracle.dequant(r["packed"], r["scale"], r["zero"], ROWS, COLS, NBITS, GROUP, AXIS)
+    dt = time.perf_counter() - t0
+    return {"value": ROWS * COLS / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "one 4096x4096 matrix of the workload, quantize+pack+dequant, "
+                      f"{dt:.1f} s single-threaded"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="own", choices=["own", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    ws, rank, local = dist_setup()
+
+    if args.impl == "reference":
+        run_reference(args, ws, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    from free_weight_quantization_b200 import hqq
+    from free_weight_quantization_b200 import workloads as wl
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        dist.init_process_group("nccl", device_id=dev,
+                                timeout=__import__("datetime").timedelta(seconds=120))
+
+    # every rank quantizes its own copies of the workload matrix
+    W0 = torch.from_numpy(wl.ATTN.make())
+    Ws = [W0.to(dev) for _ in range(ROTATE)]
+    N = ROWS * COLS
+    G = N // GROUP
+    outs = [hqq.hqq_quantize(Ws[0], NBITS, GROUP, AXIS, iters=ITERS) for _ in range(ROTATE)]
+    deqs = [torch.empty_like(Ws[0]) for _ in range(ROTATE)]
+    wsb = hqq.hqq_quantize_workspace_bytes(ROWS, COLS, NBITS, GROUP, AXIS, ITERS)
+    work = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    dbg = hqq.hqq_quantize(Ws[0], NBITS, GROUP, AXIS, iters=ITERS, debug=True)
+    torch.cuda.synchronize()
+    iters_run = int(dbg.iters_run.item())
+    rounds = int(dbg.rounds.sum().item()) if dbg.rounds is not None else None
+
+    def step(i, evs=None):
+        k = i % ROTATE
+        if evs: evs[0].record(stream)
+        hqq.hqq_quantize(Ws[k], NBITS, GROUP, AXIS, iters=ITERS, out=outs[k], workspace=work)
+        if evs: evs[1].record(stream)
+        hqq.hqq_dequantize(outs[k], out=deqs[k])
+        if evs: evs[2].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    sampler = ClockSampler(local).start()
+    time.sleep(0.3)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    tw0 = time.time()
+    start.record(stream)
+    for i in range(args.steps):
+        step(i, evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    tw1 = time.time()
+    if ws > 1:
+        dist.barrier()
+    total_ms = start.elapsed_time(end)
+    q_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    d_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+
+    # end to end through the public API: pinned host W in, packed codes + metadata + dequantized
+    # W out, copies inside the timed region
+    Wh = W0.pin_memory()
+    ph = torch.empty(outs[0].packed.numel(), dtype=torch.uint8).pin_memory()
+    sh = torch.empty(G, dtype=torch.float16).pin_memory()
+    zh = torch.empty(G, dtype=torch.float16).pin_memory()
+    dh = torch.empty(ROWS, COLS, dtype=torch.float16).pin_memory()
+    e2e_steps = max(3, min(args.steps, 50))
+
+    def e2e_step(i):
+        k = i % ROTATE
+        Ws[k].copy_(Wh, non_blocking=True)
+        hqq.hqq_quantize(Ws[k], NBITS, GROUP, AXIS, iters=ITERS, out=outs[k], workspace=work)
+        hqq.hqq_dequantize(outs[k], out=deqs[k])
+        ph.copy_(outs[k].packed, non_blocking=True)
+        sh.copy_(outs[k].scale, non_blocking=True)
+        zh.copy_(outs[k].zero, non_blocking=True)
+        dh.copy_(deqs[k], non_blocking=True)
+
+    for i in range(3):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b) / e2e_steps
+    sampler.stop()
+    clocks = sampler.summary(tw0, tw1)
+
+    # max over ranks
+    t = torch.tensor([total_ms, q_ms, d_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if ws > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, q_ms, d_ms, e2e_ms = t.tolist()
+
+    if rank == 0:
+        pk = peaks()
+        K = args.steps
+        packed_bytes = hqq.hqq_packed_bytes(N, NBITS)
+        alg_bytes = 2 * N + packed_bytes + 4 * G        # W read once; codes + fp16 meta written once
+        q_s = q_ms / 1e3 / K
+        d_s = d_ms / 1e3 / K
+        value = ws * N / q_s / 1e9
+        hbm_q = alg_bytes / q_s / 1e9
+        hbm_d = alg_bytes / d_s / 1e9
+        sm_mhz = clocks.get("sm_mhz") or pk["sm_max_mhz"]
+        alu_peak = 148 * ISSUE_LANES_PER_SM * pk["sm_max_mhz"] * 1e6 / 1e12   # T ops/s
+        roofline = None
+        if rounds is not None:
+            alg_ops = N * (ALU_OPS_INIT + ALU_OPS_FINAL) + GROUP * rounds * ALU_OPS_ROUND
+            ach = alg_ops / q_s / 1e12
+            roofline = {"bound": "alu", "kernel": "hqq_quantize (search + fixup kernels)",
+                        "achieved": ach, "peak": alu_peak, "unit": "Tops/s", "frac": ach / alu_peak,
+                        "traffic": None,
+                        "peak_src": f"148 SMs x 128 lanes x {pk['sm_max_mhz']:.0f} MHz (max clock)",
+                        "alg_ops_per_launch": alg_ops, "group_rounds": rounds}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": K,
+            "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "rows": ROWS, "cols": COLS, "nbits": NBITS,
+                       "group_size": GROUP, "axis": AXIS, "iters": ITERS,
+                       "iters_run": iters_run,
+                       "l2": f"inputs larger than L2: {ROTATE} rotating copies "
+                             f"({ROTATE * 2 * N / 1e6:.0f} MB > 126 MB)",
+                       "parallelism": f"independent matrices per rank x{ws}"},
+            "quant_us": q_s * 1e6, "dequant_us": d_s * 1e6,
+            "quant_hbm_gbs": hbm_q, "quant_hbm_frac": hbm_q / pk["hbm_gbs"],
+            "dequant_gbs": hbm_d, "dequant_hbm_frac": hbm_d / pk["hbm_gbs"],
+            "hbm_peak_gbs": pk["hbm_gbs"], "hbm_peak_src": pk["src"],
+            "alg_bytes_per_launch": alg_bytes,
+            "roofline": roofline,
+            "e2e": {"value": ws * N / (e2e_ms / 1e3) / 1e9, "unit": UNIT,
+                    "h2d_bytes_per_step": 2 * N,
+                    "d2h_bytes_per_step": packed_bytes + 4 * G + 2 * N},
+            "gpu_launches": 3 * K,
+            "clocks": clocks,
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline()
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -40,7 +40,7 @@ SIGNATURES = {
     "hqq_packed_bytes": (_I64, [_I64, _I32]),
     "hqq_quantize_workspace_bytes": (_SZ, [_I64, _I64, _I32, _I64, _I32, _I32]),
     "hqq_quantize": (_I32, [_P, _I64, _I64, _I32, _I64, _I32, ctypes.POINTER(HqqOpt), _P, _P, _P,
-                            _P, _P, _P, _P, _P, _SZ, _P]),
+                            _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "hqq_dequantize": (_I32, [_P, _P, _P, _I64, _I64, _I32, _I64, _I32, _P, _P]),
     "hqq_strerror": (ctypes.c_char_p, [_I32]),
 }
@@ -101,6 +101,7 @@ class Quantized:
     s: torch.Tensor | None = None
     z: torch.Tensor | None = None
     err_trace: torch.Tensor | None = None
+    rounds: torch.Tensor | None = None
 
 
 def hqq_quantize(W: torch.Tensor, nbits: int = 4, group_size: int = 64, axis: int = 1,
@@ -109,7 +110,8 @@ def hqq_quantize(W: torch.Tensor, nbits: int = 4, group_size: int = 64, axis: in
                  workspace: torch.Tensor | None = None, debug: bool = False,
                  stream: torch.cuda.Stream | None = None) -> Quantized:
     """HQQ quantize + pack of an fp16 CUDA matrix [rows, cols] (see hqq_quantize in the header).
-    With debug=True also returns iters_run, binary32 s and z, and the exact error trace."""
+    With debug=True also returns iters_run, binary32 s and z, the exact error trace and the
+    rounds each group needed."""
     if W.dtype != torch.float16 or not W.is_cuda or W.dim() != 2 or not W.is_contiguous():
         raise HqqError("W must be a contiguous 2-D float16 CUDA tensor")
     rows, cols = W.shape
@@ -131,6 +133,7 @@ def hqq_quantize(W: torch.Tensor, nbits: int = 4, group_size: int = 64, axis: in
             out.s = torch.empty(G, dtype=torch.float32, device=dev)
             out.z = torch.empty(G, dtype=torch.float32, device=dev)
             out.err_trace = torch.zeros(max(2 * iters, 2), dtype=torch.int64, device=dev)
+            out.rounds = torch.empty(G, dtype=torch.uint8, device=dev)
     wsb = hqq_quantize_workspace_bytes(rows, cols, nbits, group_size, axis, iters)
     if workspace is None:
         workspace = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
@@ -138,7 +141,8 @@ def hqq_quantize(W: torch.Tensor, nbits: int = 4, group_size: int = 64, axis: in
     st = stream if stream is not None else torch.cuda.current_stream(dev)
     rc = lib().hqq_quantize(_ptr(W), rows, cols, nbits, group_size, axis, ctypes.byref(opt),
                             _ptr(out.packed), _ptr(out.scale), _ptr(out.zero), _ptr(out.iters_run),
-                            _ptr(out.s), _ptr(out.z), _ptr(out.err_trace), _ptr(workspace),
+                            _ptr(out.s), _ptr(out.z), _ptr(out.err_trace), _ptr(out.rounds),
+                            _ptr(workspace),
                             workspace.numel() * workspace.element_size(),
                             ctypes.c_void_p(st.cuda_stream))
     _check(rc, "hqq_quantize")

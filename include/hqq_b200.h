@@ -97,6 +97,9 @@ size_t hqq_quantize_workspace_bytes(int64_t rows, int64_t cols, int nbits, int64
  *                over groups of floor(2^32 * sum_group |W - W_hat|) at round i, as
  *                (low 64 bits, high 64 bits); MAE_i = that / 2^32 / N.  Entries at or past
  *                iters_run are unspecified.
+ *   group_rounds [G] uint8, nullable (output): rounds each group needed before its zero
+ *                stopped moving (a later round would repeat the last one exactly), at most
+ *                iters; 0 when iters = 0.  Diagnostic: the work the loop really required.
  *   workspace    >= hqq_quantize_workspace_bytes(...) bytes, 16-byte aligned; contents on
  *                entry do not matter; must not be used by anything else until the work
  *                queued on `stream` by this call has finished
@@ -106,7 +109,7 @@ size_t hqq_quantize_workspace_bytes(int64_t rows, int64_t cols, int nbits, int64
 int hqq_quantize(const void *W, int64_t rows, int64_t cols, int nbits, int64_t group_size,
                  int axis, const hqq_opt_t *opt, void *packed, void *scale, void *zero,
                  int32_t *iters_run, float *s_f32, float *z_f32, uint64_t *err_trace,
-                 void *workspace, size_t workspace_bytes, void *stream);
+                 uint8_t *group_rounds, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Unpack + dequantize [HQQ 算法解读, "量化公式" and "从压缩文件到一次前向"]:

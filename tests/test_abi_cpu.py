@@ -73,7 +73,8 @@ def q(L, W=FAKE, rows=64, cols=64, nbits=4, g=64, axis=1, opt=None, packed=FAKE,
       zero=FAKE, ws=FAKE, wsb=1 << 20, iters_run=None):
     P = ctypes.c_void_p
     return L.hqq_quantize(P(W), rows, cols, nbits, g, axis, opt, P(packed), P(scale), P(zero),
-                          P(iters_run) if iters_run else None, None, None, None, P(ws), wsb, None)
+                          P(iters_run) if iters_run else None, None, None, None, None, P(ws), wsb,
+                          None)
 
 
 def test_quantize_rejects_on_host(L):

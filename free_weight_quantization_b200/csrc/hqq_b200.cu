@@ -34,6 +34,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <mutex>
 
 #include "hqq_b200.h"
 
@@ -1063,4 +1064,62 @@ extern "C" const char *hqq_strerror(int code) {
     case HQQ_ERR_UNSUPPORTED: return "outside this library's limits (group_size <= 256, iters <= 64)";
     default: return "unknown error";
     }
+}
+
+// ==========================================================================================
+// No-allocation variant of hqq_quantize
+//
+// Some callers cannot hand this library a workspace: code running under a host framework
+// that owns all device memory through its own pool, plugins that may not call cudaMalloc
+// (it can synchronize the device and fail once a pool has reserved the memory), or tight
+// loops that must never allocate.  For them the scratch of hqq_quantize lives in a fixed
+// buffer compiled into this library: every GPU that loads the library holds it until the
+// process exits.  Host code cannot pass the array's name to a kernel (in host code it is a
+// stand-in, not a device address), so the device address is looked up once per device with
+// cudaGetSymbolAddress while that device is current, and that address is what the kernels
+// receive.  The first call on each device does this look-up, so make that first call before
+// any stream capture.  All calls share the one buffer and it keeps the previous call's data:
+// hqq_quantize clears the part that must start at zero on every call, and two calls whose
+// work overlaps on the GPU (different streams, or different host threads) race on it.
+// ==========================================================================================
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_addr[kMaxDevices];  // device address of g_noalloc_scratch, per device
+
+int noalloc_scratch(void **out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HQQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return HQQ_ERR_CUDA;
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return HQQ_OK;
+}
+
+}  // namespace
+
+extern "C" int hqq_quantize_noalloc(const void *W, int64_t rows, int64_t cols, int nbits,
+                                    int64_t group_size, int axis, const hqq_opt_t *opt,
+                                    void *packed, void *scale, void *zero, int32_t *iters_run,
+                                    float *s_f32, float *z_f32, uint64_t *err_trace,
+                                    uint8_t *group_rounds, void *stream) {
+    hqq_opt_t o;
+    if (opt) o = *opt; else hqq_default_opt(&o);
+    Plan pl;
+    const int rc = make_plan(rows, cols, nbits, group_size, axis, o.iters, &pl);
+    if (rc != HQQ_OK) return rc;
+    if (pl.ws_total > kNoAllocScratchBytes) return HQQ_ERR_WORKSPACE;  // beyond the fixed buffer
+    void *scratch = nullptr;
+    const int sr = noalloc_scratch(&scratch);
+    if (sr != HQQ_OK) return sr;
+    return hqq_quantize(W, rows, cols, nbits, group_size, axis, &o, packed, scale, zero, iters_run,
+                        s_f32, z_f32, err_trace, group_rounds, scratch, kNoAllocScratchBytes, stream);
 }

@@ -42,6 +42,8 @@ SIGNATURES = {
     "hqq_quantize": (_I32, [_P, _I64, _I64, _I32, _I64, _I32, ctypes.POINTER(HqqOpt), _P, _P, _P,
                             _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "hqq_dequantize": (_I32, [_P, _P, _P, _I64, _I64, _I32, _I64, _I32, _P, _P]),
+    "hqq_quantize_noalloc": (_I32, [_P, _I64, _I64, _I32, _I64, _I32, ctypes.POINTER(HqqOpt), _P,
+                                    _P, _P, _P, _P, _P, _P, _P, _P]),
     "hqq_strerror": (ctypes.c_char_p, [_I32]),
 }
 
@@ -146,6 +148,34 @@ def hqq_quantize(W: torch.Tensor, nbits: int = 4, group_size: int = 64, axis: in
                             workspace.numel() * workspace.element_size(),
                             ctypes.c_void_p(st.cuda_stream))
     _check(rc, "hqq_quantize")
+    return out
+
+
+HQQ_NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def hqq_quantize_noalloc(W: torch.Tensor, nbits: int = 4, group_size: int = 64, axis: int = 1,
+                         iters: int = 20, lp_norm: float = 0.7, beta: float = 10.0,
+                         kappa: float = 1.01, eps_tiny: float = 1e-4, scale_max: float = 2e4, *,
+                         out: Quantized, stream: torch.cuda.Stream | None = None) -> Quantized:
+    """hqq_quantize for callers that cannot allocate device memory: the caller passes every
+    output buffer in `out` and the library uses its own fixed 4 MiB scratch buffer instead of a
+    workspace (see hqq_quantize_noalloc in the header).  Nothing is allocated here either."""
+    if W.dtype != torch.float16 or not W.is_cuda or W.dim() != 2 or not W.is_contiguous():
+        raise HqqError("W must be a contiguous 2-D float16 CUDA tensor")
+    rows, cols = W.shape
+    opt = HqqOpt(iters, lp_norm, beta, kappa, eps_tiny, scale_max)
+    st = stream if stream is not None else torch.cuda.current_stream(W.device)
+    rc = lib().hqq_quantize_noalloc(_ptr(W), rows, cols, nbits, group_size, axis,
+                                    ctypes.byref(opt), _ptr(out.packed), _ptr(out.scale),
+                                    _ptr(out.zero), _ptr(out.iters_run), _ptr(out.s), _ptr(out.z),
+                                    _ptr(out.err_trace), _ptr(out.rounds),
+                                    ctypes.c_void_p(st.cuda_stream))
+    if rc == 3:
+        raise HqqError("hqq_quantize_noalloc: this problem needs "
+                       f"{hqq_quantize_workspace_bytes(rows, cols, nbits, group_size, axis, iters)}"
+                       f" bytes of scratch, more than the built-in {HQQ_NOALLOC_SCRATCH_BYTES}")
+    _check(rc, "hqq_quantize_noalloc")
     return out
 
 

@@ -124,6 +124,24 @@ int hqq_dequantize(const void *packed, const void *scale, const void *zero, int6
                    int64_t cols, int nbits, int64_t group_size, int axis, void *W_out,
                    void *stream);
 
+/*
+ * hqq_quantize without a workspace argument.  The pages have no counterpart to this call: it
+ * exists for callers that cannot allocate device memory, such as plugins running inside a
+ * framework whose pool owns all of the GPU's memory, or loops that must never call cudaMalloc
+ * (it may synchronize the device).  Its scratch is a fixed 4 MiB buffer compiled into this
+ * library (HQQ_NOALLOC_SCRATCH_BYTES): every GPU that loads the library keeps it until the
+ * process exits.  Arguments, outputs and results are those of hqq_quantize; additionally it
+ * returns HQQ_ERR_WORKSPACE, launching nothing, when hqq_quantize_workspace_bytes() for these
+ * arguments exceeds that buffer.  It allocates nothing.  The first call on each device looks up
+ * the buffer's device address (make it before any stream capture).  All calls share the one
+ * buffer: calls whose GPU work overlaps (other streams, other host threads) race on it.
+ */
+#define HQQ_NOALLOC_SCRATCH_BYTES (4u << 20)
+int hqq_quantize_noalloc(const void *W, int64_t rows, int64_t cols, int nbits, int64_t group_size,
+                         int axis, const hqq_opt_t *opt, void *packed, void *scale, void *zero,
+                         int32_t *iters_run, float *s_f32, float *z_f32, uint64_t *err_trace,
+                         uint8_t *group_rounds, void *stream);
+
 /* Text for a return code (static storage). */
 const char *hqq_strerror(int code);
 

@@ -54,7 +54,7 @@ struct QParams {
     int g;          // group size
     int axis;
     int K;          // iteration cap
-    int stride;     // floats per group row in shared memory (P + 4)
+    int stride;     // floats per group row of the shared tile
     int tile;       // groups per tile
     uint8_t *packed;
     int64_t packed_bytes;
@@ -62,6 +62,8 @@ struct QParams {
     float *s_out, *z_out;
     u64 *acc;       // [K][2] direct round sums, [K][2] difference array, then control words
     uint8_t *fk;    // [G] last round run by each group in the search kernel
+    uint8_t *tile_maxf;  // [ntiles] largest f of each tile
+    int *stale;     // [ntiles] tiles holding a group whose last round lies past the kept one
     uint8_t *codes_u8;  // [N] byte-per-code staging when the packed layout is not tile aligned
     int32_t *iters_run;
     u64 *err_trace;
@@ -132,49 +134,72 @@ template <> struct Pack<2> { static constexpr int cpw = 16; };
 template <> struct Pack<3> { static constexpr int cpw = 10; };
 
 // ------------------------------------------------------------------------------------------
-// tile staging: fp16 W -> binary32 rows of the shared tile, one row of `stride` floats per
-// group [HQQ 算法解读, "`axis` 不是一个无关紧要的开关"]
+// tile staging: the tile's groups as fp16 rows of `rs` halves in shared memory
+// [HQQ 算法解读, "`axis` 不是一个无关紧要的开关"].  Each thread issues up to four 16-byte
+// loads before storing them, to keep enough bytes in flight.
 // ------------------------------------------------------------------------------------------
-__device__ void stage_tile(const QParams &P, float *wt, int64_t t0, int tg) {
-    const int g = P.g, stride = P.stride;
+__device__ void stage_tile(const QParams &P, __half *wh, int64_t t0, int tg) {
+    const int g = P.g, rs = P.stride;
     if (P.axis == 1) {
         const int ne = tg * g;
         const __half *src = P.W + t0 * (int64_t)g;  // 16-byte aligned: tiles hold 320k elements
-        const int nvec = ne >> 3;
-        for (int v = threadIdx.x; v < nvec; v += kThreads) {
-            uint4 x = __ldg(reinterpret_cast<const uint4 *>(src) + v);
-            const __half *h = reinterpret_cast<const __half *>(&x);
-            int e0 = v << 3;
-            int grp = e0 / g, j = e0 - grp * g;
+        if ((g & 7) == 0) {  // 8-element vectors never cross a row
+            const int nvec = ne >> 3;
+            for (int v0 = threadIdx.x; v0 < nvec; v0 += 4 * kThreads) {
+                uint4 x[4];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                wt[grp * stride + j] = __half2float(h[c]);
-                if (++j == g) { j = 0; ++grp; }
+                for (int u = 0; u < 4; ++u) {
+                    const int v = v0 + u * kThreads;
+                    if (v < nvec) x[u] = __ldcs(reinterpret_cast<const uint4 *>(src) + v);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int v = v0 + u * kThreads;
+                    if (v < nvec) {
+                        const int e0 = v << 3, grp = e0 / g;
+                        *reinterpret_cast<uint4 *>(wh + grp * rs + (e0 - grp * g)) = x[u];
+                    }
+                }
             }
-        }
-        for (int e = (nvec << 3) + threadIdx.x; e < ne; e += kThreads) {
-            int grp = e / g;
-            wt[grp * stride + (e - grp * g)] = __half2float(src[e]);
+        } else {
+            for (int e = threadIdx.x; e < ne; e += kThreads) {
+                const int grp = e / g;
+                wh[grp * rs + (e - grp * g)] = src[e];
+            }
         }
     } else {
         // group c of the tile is column t0 + c of the [g, G] view: elements j*G + t0 + c
         const int64_t G = P.G;
         if ((G & 7) == 0) {
             const int nv = (tg + 7) >> 3;  // tg % 8 == 0 except possibly at the end (G % 8 == 0)
-            for (int v = threadIdx.x; v < g * nv; v += kThreads) {
-                int j = v / nv, cv = v - j * nv;
-                uint4 x = __ldg(reinterpret_cast<const uint4 *>(P.W + j * G + t0) + cv);
-                const __half *h = reinterpret_cast<const __half *>(&x);
+            for (int v0 = threadIdx.x; v0 < g * nv; v0 += 4 * kThreads) {
+                uint4 x[4];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    int col = cv * 8 + c;
-                    if (col < tg) wt[col * stride + j] = __half2float(h[c]);
+                for (int u = 0; u < 4; ++u) {
+                    const int v = v0 + u * kThreads;
+                    if (v < g * nv) {
+                        const int j = v / nv, cv = v - j * nv;
+                        x[u] = __ldcs(reinterpret_cast<const uint4 *>(P.W + j * G + t0) + cv);
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int v = v0 + u * kThreads;
+                    if (v < g * nv) {
+                        const int j = v / nv, cv = v - j * nv;
+                        const __half *h = reinterpret_cast<const __half *>(&x[u]);
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            const int col = cv * 8 + c;
+                            if (col < tg) wh[col * rs + j] = h[c];
+                        }
+                    }
                 }
             }
         } else {
             for (int v = threadIdx.x; v < g * tg; v += kThreads) {
-                int j = v / tg, col = v - j * tg;
-                wt[col * stride + j] = __half2float(P.W[j * G + t0 + col]);
+                const int j = v / tg, col = v - j * tg;
+                wh[col * rs + j] = P.W[j * G + t0 + col];
             }
         }
     }
@@ -184,77 +209,84 @@ __device__ void stage_tile(const QParams &P, float *wt, int64_t t0, int tg) {
 // Also keeps W*s of the group's min and max element: every element's W*s lies between them
 // (rounding is monotonic), which bounds W*s + z without visiting the elements.
 template <int NB>
-__device__ void init_tile(const QParams &P, const float *wt, float *s_t, float *z_t, float *lo_t,
+__device__ void init_tile(const QParams &P, const __half *wh, float *s_t, float *z_t, float *lo_t,
                           float *hi_t, int tg) {
     constexpr float kQmax = (float)((1 << NB) - 1);
+    const int g = P.g;
     for (int i = threadIdx.x; i < tg; i += kThreads) {
-        const float *row = wt + i * P.stride;
-        float mn = row[0], mx = row[0];
-        for (int j = 1; j < P.g; ++j) {
-            mn = fminf(mn, row[j]);
-            mx = fmaxf(mx, row[j]);
+        const __half *row = wh + i * P.stride;
+        float mn[4], mx[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) { mn[c] = INFINITY; mx[c] = -INFINITY; }
+        int j = 0;
+        for (; j + 4 <= g; j += 4) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float v = __half2float(row[j + c]);
+                mn[c] = fminf(mn[c], v);
+                mx[c] = fmaxf(mx[c], v);
+            }
         }
-        float d = __fsub_rn(mx, mn);
+        for (; j < g; ++j) {
+            const float v = __half2float(row[j]);
+            mn[0] = fminf(mn[0], v);
+            mx[0] = fmaxf(mx[0], v);
+        }
+        const float lo_w = fminf(fminf(mn[0], mn[1]), fminf(mn[2], mn[3]));
+        const float hi_w = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        const float d = __fsub_rn(hi_w, lo_w);
         float s = (d < P.eps_tiny) ? 1.0f : __fdiv_rn(kQmax, d);
         s = fminf(s, P.scale_max);
         s_t[i] = s;
-        z_t[i] = __fsub_rn(0.0f, __fmul_rn(mn, s));
-        lo_t[i] = __fmul_rn(mn, s);
-        hi_t[i] = __fmul_rn(mx, s);
+        z_t[i] = __fsub_rn(0.0f, __fmul_rn(lo_w, s));
+        lo_t[i] = __fmul_rn(lo_w, s);
+        hi_t[i] = __fmul_rn(hi_w, s);
     }
 }
 
-// ------------------------------------------------------------------------------------------
-// the proximal loop [HQQ 算法解读, "第二拍：half-quadratic 迭代修正零点"]
-//
-// The CTA advances its tile round by round.  A list in shared memory holds the groups that
-// are still active; each pass of a warp takes NSEG of them (one per segment of L lanes), so
-// finished groups drop out and the remaining ones are packed onto as few warps as possible.
-// Within a round every contribution goes to the same round index, which lets a warp add its
-// segments' errors with native 32-bit reductions (16-bit chunks of the 64-bit fixed-point
-// value) before one shared-memory add.
-//
-// REPLAY = false (search): a group leaves the list once frozen (z_{r+1} == z_r, no residual
-//   above the last round's shrink threshold: every later round repeats round r exactly) or
-//   after round K-1; its codes for z_r stay in its tile row and f_t = r.  Per-round error
-//   sums go to acc_c[0][r]; a group frozen at r also adds its error to acc_c[1][r+1] (a
-//   difference array: that error repeats in every later round).
-// REPLAY = true (fixup): a group makes exactly n = min(b, f_t) zero updates and leaves its
-//   codes for z_n in its tile row.
-// ------------------------------------------------------------------------------------------
-__device__ __forceinline__ void warp_add_fixed(unsigned *dst, u64 v) {
-    // exact sum over the warp of 64-bit values, as four 16-bit chunks (each chunk sum < 2^21)
-    const unsigned c0 = __reduce_add_sync(kFull, (unsigned)(v & 0xffffu));
-    const unsigned c1 = __reduce_add_sync(kFull, (unsigned)((v >> 16) & 0xffffu));
-    const unsigned c2 = __reduce_add_sync(kFull, (unsigned)((v >> 32) & 0xffffu));
-    const unsigned c3 = __reduce_add_sync(kFull, (unsigned)(v >> 48));
-    if ((threadIdx.x & 31) == 0) {  // the row belongs to this warp alone
-        dst[0] += c0;
-        dst[1] += c1;
-        dst[2] += c2;
-        dst[3] += c3;
+// Code storage of a lane's 16 codes while the group iterates.  DIRECT: already in the packed
+// format of the output (4 bit: two words of eight nibbles; 2 bit: one word), written straight
+// to global memory when the group is done.  Otherwise one byte per code, left in the tile row
+// and packed when the tile is written out.
+template <int NB, bool DIRECT>
+struct Codes {
+    static constexpr int kWords = DIRECT ? (NB == 4 ? 2 : 1) : 4;
+    static constexpr int kBits = DIRECT ? NB : 8;
+    uint32_t w[kWords];
+    __device__ __forceinline__ void put(int m, uint32_t bits) {
+        // insert the low NB bits of `bits` at the code's position
+        constexpr int per = 32 / kBits;
+        uint32_t d;
+        asm("bfi.b32 %0, %1, %2, %3, %4;" : "=r"(d)
+            : "r"(bits), "r"(m % per == 0 ? 0u : w[m / per]), "r"(kBits * (m % per)), "r"(NB));
+        w[m / per] = d;
     }
-}
+};
 
 // One round over the 16 elements a lane holds: t = W*s + z, q = round(clip(t)), W_hat from
-// the code table, |W - W_hat| and q - W*s (the zero-update term with e = 0).  CLIP = false
-// is used only when every t of the warp's groups is known to round inside [0, 2^b - 1].
-template <int NB, int NSEG, bool CLIP, bool FULL>
-__device__ __forceinline__ void round_elems(const float (&w)[kE], float s, float z,
-                                            const float *tab, int sg, int nvalid,
-                                            float (&absr)[kE], float (&term)[kE]) {
+// the code table, |W - W_hat| and q - W*s (the zero-update term with e = 0); the codes are
+// kept.  CLIP = false only when every t of the warp's groups rounds inside [0, 2^b - 1].
+template <int NB, int NSEG, bool CLIP, bool FULL, bool DIRECT>
+__device__ __forceinline__ void round_elems(const float (&w)[kE], const float (&ws)[kE], float z,
+                                            uint32_t tab_adj, int nvalid, float (&absr)[kE],
+                                            float (&term)[kE], Codes<NB, DIRECT> &codes) {
     constexpr int NQ = 1 << NB;
     constexpr float kQmax = (float)(NQ - 1);
+    constexpr int kShift = NSEG == 32 ? 7 : NSEG == 16 ? 6 : NSEG == 8 ? 5 : NSEG == 4 ? 4 : 3;
 #pragma unroll
     for (int m = 0; m < kE; ++m) {
-        const float wsm = __fmul_rn(w[m], s);
-        float t = __fadd_rn(wsm, z);
+        float t = __fadd_rn(ws[m], z);
         if (CLIP) t = fminf(fmaxf(t, 0.0f), kQmax);  // clip then round == round then clip
         const float u = __fadd_rn(t, kMagic);
         const float qf = __fsub_rn(u, kMagic);        // round half to even
-        const float what = tab[(__float_as_int(u) & (NQ - 1)) * NSEG + sg];
+        // u's bit pattern is 0x4B400000 + q: the table entry of code q sits at
+        // tab_adj + (bits << kShift) (mod 2^32), tab_adj having absorbed the constant part
+        const uint32_t bits = __float_as_uint(u);
+        float what;
+        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(what) : "r"(tab_adj + (bits << kShift)));
+        codes.put(m, bits);
         const float ar = fabsf(__fsub_rn(w[m], what));
-        const float tm = __fsub_rn(qf, wsm);          // q - (W - 0)*s
+        const float tm = __fsub_rn(qf, ws[m]);        // q - (W - 0)*s
         if (FULL) {
             absr[m] = ar;
             term[m] = tm;
@@ -265,77 +297,138 @@ __device__ __forceinline__ void round_elems(const float (&w)[kE], float s, float
     }
 }
 
-// Each warp owns a contiguous slice of at most 64 groups of the tile and runs its rounds on
-// its own (no block-wide barrier inside the loop).  The slice's active groups are the set
-// bits of a 64-bit mask, listed in shared memory at the start of each round; a pass hands
-// the next NSEG of them to the warp's segments.
-template <int NB, int L, bool REPLAY, bool FULL>
-__device__ void run_rounds(const QParams &P, const float *wt, const float *s_t, float *z_t,
+__device__ __forceinline__ void add_fixed(unsigned *row, u64 v) {
+    // 64-bit fixed-point value into four 16-bit-chunk counters (exact; no counter overflows)
+    atomicAdd(row, (unsigned)(v & 0xffffu));
+    atomicAdd(row + 1, (unsigned)((v >> 16) & 0xffffu));
+    atomicAdd(row + 2, (unsigned)((v >> 32) & 0xffffu));
+    atomicAdd(row + 3, (unsigned)(v >> 48));
+}
+
+// metadata of one group [HQQ 算法解读, "量化公式"]: Delta = 1/s and z, rounded to fp16
+__device__ __forceinline__ void write_meta(const QParams &P, int64_t k, float s, float z, int f) {
+    P.scale[k] = __float2half_rn(__fdiv_rn(1.0f, s));
+    P.zero[k] = __float2half_rn(z);
+    if (P.s_out) P.s_out[k] = s;
+    if (P.z_out) P.z_out[k] = z;
+    if (f >= 0) {
+        P.fk[k] = (uint8_t)f;
+        if (P.group_rounds) P.group_rounds[k] = P.K > 0 ? (uint8_t)(f + 1) : 0;
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// the proximal loop [HQQ 算法解读, "第二拍：half-quadratic 迭代修正零点"]
+//
+// Each warp owns a contiguous slice of the tile's groups.  A segment of L lanes takes the
+// slice's next group, keeps its 16-element runs in registers (binary32) and runs round after
+// round until the group is done, then takes the next one, so lanes never idle while the
+// slice has work left.  Segments of a warp may be at different rounds.
+//   search (REPLAY = false): a group is done once frozen (z_{r+1} == z_r and no residual
+//     above the last round's shrink threshold: every later round repeats round r exactly) or
+//     after round K-1.  Round r's error is added to counters acc_w[r]; a group frozen at r
+//     also adds it to acc_w[K + r + 1] (a difference array: it repeats in every later round).
+//   fixup (REPLAY = true): a group makes exactly n = min(b, f) zero updates.
+// The codes of a group's last round are its final codes (the final quantize with the
+// original W and the kept zero, section "第二拍"): a done group writes them, with its
+// metadata, straight to global memory (DIRECT) or leaves them in its tile row.
+// ------------------------------------------------------------------------------------------
+template <int NB, int L, bool REPLAY, bool FULL, bool DIRECT>
+__device__ void run_groups(const QParams &P, __half *wh, const float *s_t, float *z_t,
                            const float *lo_t, const float *hi_t, uint8_t *f_t, float *tab,
-                           uint8_t *list, unsigned *acc_w, int tg, int b_stop) {
+                           unsigned *acc_w, const float *thr_s, const double *beta_s, int64_t t0,
+                           int tg, int b_stop) {
     constexpr int NQ = 1 << NB;
     constexpr float kQmax = (float)(NQ - 1);
     constexpr int NSEG = 32 / L;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int sg = lane / L, l = lane - sg * L;
     const unsigned seg_mask = (L == 32) ? kFull : (((1u << L) - 1u) << (sg * L));
-    const int K = P.K, stride = P.stride;
+    const int K = P.K, rs = P.stride;
     const int nvalid = FULL ? kE : min(max(P.g - l * kE, 0), kE);
     const float g_f = (float)P.g, inv_g = 1.0f / (float)P.g;  // exact for FULL (g = 2^k)
-    const float thr_last = K > 0 ? P.thr[K - 1] : 0.0f;
-    const int rounds = REPLAY ? b_stop : K;
-    const int gpw = (P.tile + kWarps - 1) / kWarps;  // <= 64 (host plan)
+    const float thr_last = K > 0 ? thr_s[K - 1] : 0.0f;
+    const int gpw = (P.tile + kWarps - 1) / kWarps;
     const int g0 = warp * gpw;
     const int ng = max(0, min(gpw, tg - g0));
+    const float lf = (float)l;  // code k = l + kk*L of the table, as an exact float
+    // shared-space address of this segment's table column, minus the contribution of the
+    // constant high bits of a rounded value (see round_elems); wraps modulo 2^32 on purpose
+    constexpr int kShift = NSEG == 32 ? 7 : NSEG == 16 ? 6 : NSEG == 8 ? 5 : NSEG == 4 ? 4 : 3;
+    const uint32_t tab_adj = (uint32_t)__cvta_generic_to_shared(tab + sg) - (0x4B400000u << kShift);
 
-    u64 mask = 0;
-    for (int gi = lane; gi < ng; gi += 32) {
-        const bool go = REPLAY ? (min(b_stop, (int)f_t[g0 + gi]) > 0) : (K > 0);
-        if (go) mask |= 1ull << gi;
-        else if (!REPLAY) f_t[g0 + gi] = 0;
-    }
-    mask = ((u64)__reduce_or_sync(kFull, (unsigned)(mask >> 32)) << 32) |
-           __reduce_or_sync(kFull, (unsigned)mask);
-
-    for (int r = 0; r < rounds && mask; ++r) {
-        const int n_act = __popcll(mask);
-        __syncwarp();
-        for (int i = lane; i < 64; i += 32)
-            if ((mask >> i) & 1ull) list[__popcll(mask & ((1ull << i) - 1ull))] = (uint8_t)i;
-        __syncwarp();
-        const float thr_r = P.thr[r];
-        u64 fx_acc = 0, fd_acc = 0, dmask = 0;
-        for (int base = 0; base < n_act; base += NSEG) {
-            const int idx = base + sg;
-            const bool active = idx < n_act;
-            const int gi = list[active ? idx : base];
-            const int grp = g0 + gi;
-            float w[kE];
-            const float4 *src = reinterpret_cast<const float4 *>(wt + grp * stride + l * kE);
+    // Every lane's state stays in range even with no group: the table address of round_elems
+    // assumes W*s + z rounds inside [0, 2^b - 1] whenever the clip is skipped
+    float w[kE], ws[kE];
 #pragma unroll
-            for (int v = 0; v < kE / 4; ++v) {
-                const float4 x = src[v];
-                w[4 * v] = x.x; w[4 * v + 1] = x.y; w[4 * v + 2] = x.z; w[4 * v + 3] = x.w;
+    for (int m = 0; m < kE; ++m) { w[m] = 0.0f; ws[m] = 0.0f; }
+    float s = 1.0f, z = 0.0f, lo = 0.0f, hi = 0.0f;
+    int grp = -1, it = 0, nupd = 0, next = 0;
+    bool exhausted = false;
+    Codes<NB, DIRECT> codes;
+#pragma unroll
+    for (int i = 0; i < Codes<NB, DIRECT>::kWords; ++i) codes.w[i] = 0;
+    while (true) {
+        // ---- refill: segments without a group take the slice's next ones in lane order
+        const bool need = grp < 0 && !exhausted;
+        if (__any_sync(kFull, need)) {
+            const unsigned nm = __ballot_sync(kFull, need && l == 0);
+            int cand = next + __popc(nm & ((1u << lane) - 1u));
+            cand = __shfl_sync(kFull, cand, sg * L);
+            next += __popc(nm);
+            if (need) {
+                if (cand < ng) {
+                    grp = g0 + cand;
+                    const uint4 *src = reinterpret_cast<const uint4 *>(wh + grp * rs + l * kE);
+                    const uint4 a = src[0], b = src[1];
+                    const __half2 *ha = reinterpret_cast<const __half2 *>(&a);
+                    const __half2 *hb = reinterpret_cast<const __half2 *>(&b);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float2 x = __half22float2(ha[i]), y = __half22float2(hb[i]);
+                        w[2 * i] = x.x; w[2 * i + 1] = x.y; w[8 + 2 * i] = y.x; w[9 + 2 * i] = y.y;
+                    }
+                    s = s_t[grp];
+                    z = z_t[grp];
+                    lo = lo_t[grp];
+                    hi = hi_t[grp];
+#pragma unroll
+                    for (int m = 0; m < kE; ++m) ws[m] = __fmul_rn(w[m], s);
+                    if (!FULL) {  // slots past the group's end: W*s at the group's minimum
+#pragma unroll
+                        for (int m = 0; m < kE; ++m)
+                            if (m >= nvalid) { w[m] = 0.0f; ws[m] = lo; }
+                    }
+                    it = 0;
+                    if (REPLAY) nupd = min(b_stop, (int)f_t[grp]);
+                } else {
+                    exhausted = true;
+                }
             }
-            const float s = s_t[grp];
-            const float z = z_t[grp];
-            // t of every element of the group lies in [lo + z, hi + z]: no clip is needed when
-            // that range rounds inside [0, 2^b - 1]
-            const bool inside = __fadd_rn(lo_t[grp], z) >= -0.5f && __fadd_rn(hi_t[grp], z) < kQmax + 0.5f;
-            const bool noclip = __all_sync(kFull, inside);
+        }
+        const bool active = grp >= 0;
+        if (!__any_sync(kFull, active)) break;
 
+        const bool do_iter = active && (REPLAY ? (it < nupd) : (K > 0));
+        bool done = active && !do_iter;
+        if (__any_sync(kFull, do_iter)) {
+            const int ri = min(it, max(K - 1, 0));
+            // no clip is needed when [lo + z, hi + z] rounds inside [0, 2^b - 1]; lanes
+            // without a group keep their last group's (or zero) state, so they are tested too
+            const bool inside = __fadd_rn(lo, z) >= -0.5f && __fadd_rn(hi, z) < kQmax + 0.5f;
+            const bool noclip = __all_sync(kFull, inside);
             // reconstructions W_hat = (k - z)/s for every code k: the IEEE division of the
             // method, done once per code value instead of once per element
             __syncwarp();
 #pragma unroll
             for (int kk = 0; kk < (NQ + L - 1) / L; ++kk) {
                 const int k = l + kk * L;
-                if (k < NQ) tab[k * NSEG + sg] = __fdiv_rn(__fsub_rn((float)k, z), s);
+                if (k < NQ) tab[k * NSEG + sg] = __fdiv_rn(__fsub_rn(lf + (float)(kk * L), z), s);
             }
             __syncwarp();
             float absr[kE], term[kE];
-            if (noclip) round_elems<NB, NSEG, false, FULL>(w, s, z, tab, sg, nvalid, absr, term);
-            else round_elems<NB, NSEG, true, FULL>(w, s, z, tab, sg, nvalid, absr, term);
+            if (noclip) round_elems<NB, NSEG, false, FULL, DIRECT>(w, ws, z, tab_adj, nvalid, absr, term, codes);
+            else round_elems<NB, NSEG, true, FULL, DIRECT>(w, ws, z, tab_adj, nvalid, absr, term, codes);
             const float esum_l = tree16(absr);
             // the lane's largest residual is at most its partial sum; only when that bound
             // fails is the maximum taken
@@ -348,12 +441,12 @@ __device__ void run_rounds(const QParams &P, const float *wt, const float *s_t, 
             const float esum = seg_sum<L>(esum_l);
             float zsum = seg_sum<L>(tree16(term));
             // lp shrink: a residual above the round's safe threshold -> exact binary64 path
-            const bool slow = (__ballot_sync(kFull, active && maxr > thr_r) & seg_mask) != 0;
+            const bool slow = (__ballot_sync(kFull, do_iter && maxr > thr_s[ri]) & seg_mask) != 0;
             if (__any_sync(kFull, slow)) {
-                const double beta = P.beta[r];
+                const double beta = beta_s[ri];
 #pragma unroll
                 for (int m = 0; m < kE; ++m) {
-                    float t = __fadd_rn(__fmul_rn(w[m], s), z);
+                    float t = __fadd_rn(ws[m], z);
                     t = fminf(fmaxf(t, 0.0f), kQmax);
                     const float u = __fadd_rn(t, kMagic);
                     const float qf = __fsub_rn(u, kMagic);
@@ -366,110 +459,89 @@ __device__ void run_rounds(const QParams &P, const float *wt, const float *s_t, 
                 if (slow) zsum = zs2;
             }
             const float znew = FULL ? __fmul_rn(zsum, inv_g) : __fdiv_rn(zsum, g_f);
-
-            bool done;
-            float zfin;
-            if (!REPLAY) {
-                const bool big = (__ballot_sync(kFull, maxr > thr_last) & seg_mask) != 0;
-                const bool frozen = !slow && !big && (znew == z);
-                done = frozen || r == K - 1;
-                zfin = z;
-                if (active && l == 0) {
-                    const u64 fx = err_fixed(esum);
-                    fx_acc += fx;
-                    if (done && r + 1 < K) fd_acc += fx;
+            const bool big = (__ballot_sync(kFull, maxr > thr_last) & seg_mask) != 0;
+            if (do_iter) {
+                if (!REPLAY) {
+                    const bool frozen = !slow && !big && (znew == z);
+                    done = frozen || it == K - 1;
+                    if (l == 0) {
+                        const u64 fx = err_fixed(esum);
+                        add_fixed(acc_w + 4 * it, fx);
+                        if (done && it + 1 < K) add_fixed(acc_w + 4 * (K + it + 1), fx);
+                    }
+                    if (!done) {
+                        z = znew;
+                        ++it;
+                    }
+                } else {
+                    z = znew;
+                    ++it;
+                    done = it >= nupd;
                 }
+            }
+        }
+        if (done) {
+            if (REPLAY || K == 0) {
+                // replay: the last round's codes were for z_{n-1}, the kept zero is z_n; no
+                // round at all: codes for z0.  Either way quantize once more here.
+#pragma unroll
+                for (int m = 0; m < kE; ++m) {
+                    const float t = fminf(fmaxf(__fadd_rn(ws[m], z), 0.0f), kQmax);
+                    codes.put(m, __float_as_uint(__fadd_rn(t, kMagic)));
+                }
+            }
+            const int64_t kg = t0 + grp;
+            if (DIRECT) {
+                if (nvalid > 0) {
+                    const int64_t e = kg * P.g + l * kE;  // flat index of the lane's first code
+                    if (NB == 4)
+                        *reinterpret_cast<uint2 *>(P.packed + e / 2) = make_uint2(codes.w[0], codes.w[1]);
+                    else
+                        *reinterpret_cast<uint32_t *>(P.packed + e / 4) = codes.w[0];
+                }
+                if (l == 0) write_meta(P, kg, s, z, REPLAY ? -1 : it);
             } else {
-                done = r + 1 >= min(b_stop, (int)f_t[grp]);
-                zfin = znew;
-            }
-            if (active && l == 0) {
-                z_t[grp] = done ? zfin : znew;
-                if (done) {
-                    if (!REPLAY) f_t[grp] = (uint8_t)r;
-                    dmask |= 1ull << gi;
+                // the row's halves are dead (the group lives in registers): its bytes take the codes
+                *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(wh + grp * rs) + l * kE) =
+                    make_uint4(codes.w[0], codes.w[1 % Codes<NB, DIRECT>::kWords],
+                               codes.w[2 % Codes<NB, DIRECT>::kWords],
+                               codes.w[3 % Codes<NB, DIRECT>::kWords]);
+                if (l == 0) {
+                    z_t[grp] = z;
+                    if (!REPLAY) f_t[grp] = (uint8_t)it;
                 }
             }
+            grp = -1;
         }
-        if (!REPLAY) {
-            warp_add_fixed(acc_w + 4 * r, fx_acc);
-            if (r + 1 < K) warp_add_fixed(acc_w + 4 * (K + r + 1), fd_acc);
-        }
-        dmask = ((u64)__reduce_or_sync(kFull, (unsigned)(dmask >> 32)) << 32) |
-                __reduce_or_sync(kFull, (unsigned)dmask);
-        mask &= ~dmask;
     }
 }
 
 // ------------------------------------------------------------------------------------------
-// tile output: metadata [HQQ 算法解读, "量化公式"] and packed codes [HQQ 算法解读, "为什么一定要分组"]
-// The final quantize with the original W and the kept z (section "第二拍") happens here: step 1
-// turns each 16-element run of a group row into codes in a byte buffer laid out in flat
-// tensor order for the tile; step 2 packs that buffer into 32-bit words.
+// tile output when codes are not written directly: metadata [HQQ 算法解读, "量化公式"] and
+// packed codes [HQQ 算法解读, "为什么一定要分组"] from the code bytes at the start of each row
 // ------------------------------------------------------------------------------------------
 template <int NB>
-__device__ void write_tile(const QParams &P, const float *wt, const float *s_t, const float *z_t,
-                           uint8_t *cbuf, int64_t t0, int tg) {
-    constexpr float kQmax = (float)((1 << NB) - 1);
-    for (int i = threadIdx.x; i < tg; i += kThreads) {
-        const int64_t k = t0 + i;
-        const float s = s_t[i], z = z_t[i];
-        P.scale[k] = __float2half_rn(__fdiv_rn(1.0f, s));
-        P.zero[k] = __float2half_rn(z);
-        if (P.s_out) P.s_out[k] = s;
-        if (P.z_out) P.z_out[k] = z;
-    }
-    const int g = P.g, stride = P.stride;
-    const int L = (P.stride - 4) / kE;  // lanes per group row (P / 16)
-    // step 1: codes
-    for (int it = threadIdx.x; it < tg * L; it += kThreads) {
-        const int grp = it / L, l = it - grp * L;
-        const int j0 = l * kE;
-        if (j0 >= g) continue;
-        const float s = s_t[grp], z = z_t[grp];
-        const float4 *src = reinterpret_cast<const float4 *>(wt + grp * stride + j0);
-        uint32_t qw[kE / 4];  // codes, four per word, lowest index in the lowest byte
-#pragma unroll
-        for (int v = 0; v < kE / 4; ++v) {
-            const float4 x = src[v];
-            const float xs[4] = {x.x, x.y, x.z, x.w};
-            uint32_t word = 0;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float t = fminf(fmaxf(__fadd_rn(__fmul_rn(xs[c], s), z), 0.0f), kQmax);
-                word |= (uint32_t)(__float_as_int(__fadd_rn(t, kMagic)) & ((1 << NB) - 1)) << (8 * c);
-            }
-            qw[v] = word;
-        }
-        const int n = min(kE, g - j0);
-        if (P.axis == 1) {
-            uint8_t *dst = cbuf + grp * g + j0;
-            if (n == kE && ((grp * g + j0) & 15) == 0) {
-                *reinterpret_cast<uint4 *>(dst) = make_uint4(qw[0], qw[1], qw[2], qw[3]);
-            } else {
-#pragma unroll
-                for (int m = 0; m < kE; ++m)
-                    if (m < n) dst[m] = (uint8_t)(qw[m / 4] >> (8 * (m % 4)));
-            }
-        } else {
-#pragma unroll
-            for (int m = 0; m < kE; ++m)
-                if (m < n) cbuf[(j0 + m) * tg + grp] = (uint8_t)(qw[m / 4] >> (8 * (m % 4)));
-        }
-    }
-    __syncthreads();
+__device__ void write_tile(const QParams &P, const __half *wh, const float *s_t,
+                           const float *z_t, const uint8_t *f_t, bool search, int64_t t0, int tg) {
+    for (int i = threadIdx.x; i < tg; i += kThreads)
+        write_meta(P, t0 + i, s_t[i], z_t[i], search ? (int)f_t[i] : -1);
+    const int g = P.g;
+    const int rowb = 2 * P.stride;  // bytes per tile row
+    const uint8_t *cb = reinterpret_cast<const uint8_t *>(wh);
     if (P.codes_u8) {  // byte-per-code staging, packed afterwards by pack_codes_kernel
         if (P.axis == 1) {
-            for (int e = threadIdx.x; e < tg * g; e += kThreads) P.codes_u8[t0 * g + e] = cbuf[e];
+            for (int e = threadIdx.x; e < tg * g; e += kThreads) {
+                const int grp = e / g;
+                P.codes_u8[t0 * g + e] = cb[grp * rowb + (e - grp * g)];
+            }
         } else {
             for (int v = threadIdx.x; v < tg * g; v += kThreads) {
                 const int j = v / tg, col = v - j * tg;
-                P.codes_u8[j * P.G + t0 + col] = cbuf[v];
+                P.codes_u8[j * P.G + t0 + col] = cb[col * rowb + j];
             }
         }
         return;
     }
-    // step 2: words of CPW codes from the flat code buffer
     constexpr int CPW = Pack<NB>::cpw;
     auto store_word = [&](int64_t widx, uint32_t word) {
         const int64_t off = widx * 4;
@@ -480,80 +552,93 @@ __device__ void write_tile(const QParams &P, const float *wt, const float *s_t, 
                 if (off + b < P.packed_bytes) P.packed[off + b] = (uint8_t)(word >> (8 * b));
         }
     };
-    auto pack_word = [&](const uint8_t *c, int n) -> uint32_t {
-        uint32_t word = 0;
-#pragma unroll
-        for (int k = 0; k < CPW; ++k)
-            if (k < n) word |= (uint32_t)c[k] << (NB * k);
-        return word;
-    };
     if (P.axis == 1) {
         const int ne = tg * g;
         const int nw = (ne + CPW - 1) / CPW;
         const int64_t w0 = t0 * g / CPW;  // tiles start on a word boundary
-        for (int wi = threadIdx.x; wi < nw; wi += kThreads)
-            store_word(w0 + wi, pack_word(cbuf + wi * CPW, min(CPW, ne - wi * CPW)));
+        for (int wi = threadIdx.x; wi < nw; wi += kThreads) {
+            const int e0 = wi * CPW;
+            int grp = e0 / g, j = e0 - grp * g;
+            uint32_t word = 0;
+#pragma unroll
+            for (int k = 0; k < CPW; ++k) {
+                if (e0 + k < ne) {
+                    word |= (uint32_t)cb[grp * rowb + j] << (NB * k);
+                    if (++j == g) { j = 0; ++grp; }
+                }
+            }
+            store_word(w0 + wi, word);
+        }
     } else {
         // row j of the [g, G] view holds the tile's codes at flat j*G + t0 + col; here
         // G % CPW == 0 and t0 % CPW == 0, so each row segment starts on a word boundary
         const int nwr = (tg + CPW - 1) / CPW;
         for (int v = threadIdx.x; v < g * nwr; v += kThreads) {
             const int j = v / nwr, wr = v - j * nwr;
-            store_word((j * P.G + t0) / CPW + wr,
-                       pack_word(cbuf + j * tg + wr * CPW, min(CPW, tg - wr * CPW)));
+            uint32_t word = 0;
+#pragma unroll
+            for (int k = 0; k < CPW; ++k) {
+                const int col = wr * CPW + k;
+                if (col < tg) word |= (uint32_t)cb[col * rowb + j] << (NB * k);
+            }
+            store_word((j * P.G + t0) / CPW + wr, word);
         }
     }
 }
 
 struct SmemLayout {
-    int wt, s_t, z_t, lo_t, hi_t, f_t, tab, list, acc, cbuf, total;
+    int wh, s_t, z_t, lo_t, hi_t, f_t, tab, acc, thr, beta, total;
 };
 
-__host__ __device__ inline SmemLayout smem_layout(int tile, int stride, int nq, int L, int K) {
+__host__ __device__ inline SmemLayout smem_layout(int tile, int rs, int nq, int L, int K) {
     SmemLayout s;
+    const int Kc = K > 0 ? K : 1;
     int o = 0;
-    s.wt = o; o += tile * stride * 4;
+    s.wh = o; o += (tile * rs * 2 + 15) / 16 * 16;
     s.s_t = o; o += tile * 4;
     s.z_t = o; o += tile * 4;
     s.lo_t = o; o += tile * 4;
     s.hi_t = o; o += tile * 4;
     s.f_t = o; o += (tile + 15) / 16 * 16;
     s.tab = o; o += kWarps * nq * (32 / L) * 4;
-    s.list = o; o += kWarps * 64;
-    s.acc = o; o += kWarps * 2 * (K > 0 ? K : 1) * 4 * 4;  // per warp: [2][K] x 4 chunks
-    s.cbuf = o; o += (tile * (stride - 4) + 15) / 16 * 16;  // codes of the tile, one byte each
+    s.acc = o; o += kWarps * 2 * Kc * 4 * 4;  // per warp: [2][K] x 4 chunks
+    s.thr = o; o += (Kc * 4 + 15) / 16 * 16;
+    s.beta = o; o += Kc * 8;
     s.total = o;
     return s;
 }
 
 template <int NB, int L>
 struct Smem {
-    float *wt, *s_t, *z_t, *lo_t, *hi_t, *tab;
-    uint8_t *f_t, *list, *cbuf;
-    unsigned *acc;  // all warps' rows
-    unsigned *acc_w;  // this warp's row
+    __half *wh;
+    float *s_t, *z_t, *lo_t, *hi_t, *tab, *thr;
+    double *beta;
+    uint8_t *f_t;
+    unsigned *acc;    // all warps' counters
+    unsigned *acc_w;  // this warp's counters
     __device__ Smem(unsigned char *base, const QParams &P) {
         const SmemLayout lay = smem_layout(P.tile, P.stride, 1 << NB, L, P.K);
-        wt = reinterpret_cast<float *>(base + lay.wt);
+        wh = reinterpret_cast<__half *>(base + lay.wh);
         s_t = reinterpret_cast<float *>(base + lay.s_t);
         z_t = reinterpret_cast<float *>(base + lay.z_t);
         lo_t = reinterpret_cast<float *>(base + lay.lo_t);
         hi_t = reinterpret_cast<float *>(base + lay.hi_t);
         f_t = base + lay.f_t;
-        list = base + lay.list + (threadIdx.x >> 5) * 64;
-        cbuf = base + lay.cbuf;
         tab = reinterpret_cast<float *>(base + lay.tab) + (threadIdx.x >> 5) * (1 << NB) * (32 / L);
         acc = reinterpret_cast<unsigned *>(base + lay.acc);
         acc_w = acc + (threadIdx.x >> 5) * 8 * (P.K > 0 ? P.K : 1);
+        thr = reinterpret_cast<float *>(base + lay.thr);
+        beta = reinterpret_cast<double *>(base + lay.beta);
     }
 };
 
-// workspace words after the per-round sums: tiles finished, kept round, rounds measured
+// workspace words after the per-round sums: tiles finished, kept round, rounds measured,
+// number of stale tiles; then the per-tile largest f and the list of stale tiles
 struct Ctl {
     unsigned done;
     int b;
     int run;
-    int pad;
+    int nstale;
 };
 
 __device__ __forceinline__ Ctl *ctl_of(const QParams &P) {
@@ -592,27 +677,38 @@ __device__ void stop_rule(const QParams &P) {
     if (P.iters_run) *P.iters_run = run;
 }
 
-template <int NB, int L, bool FULL>
-__global__ void __launch_bounds__(kThreads) hqq_search_kernel(const __grid_constant__ QParams P) {
+template <int NB, int L>
+__device__ void load_constants(const QParams &P, Smem<NB, L> &S) {
+    for (int i = threadIdx.x; i < P.K; i += kThreads) {
+        S.thr[i] = P.thr[i];
+        S.beta[i] = P.beta[i];
+    }
+}
+
+template <int NB, int L, bool FULL, bool DIRECT>
+__global__ void __launch_bounds__(kThreads, 2) hqq_search_kernel(const __grid_constant__ QParams P) {
     extern __shared__ __align__(16) unsigned char smem[];
     Smem<NB, L> S(smem, P);
     __shared__ bool last;
+    __shared__ int maxf;
     const int K = P.K;
     const int64_t t0 = (int64_t)blockIdx.x * P.tile;
     const int tg = (int)min((int64_t)P.tile, P.G - t0);
     for (int i = threadIdx.x; i < kWarps * 8 * K; i += kThreads) S.acc[i] = 0;
-    stage_tile(P, S.wt, t0, tg);
+    if (threadIdx.x == 0) maxf = 0;
+    load_constants(P, S);
+    stage_tile(P, S.wh, t0, tg);
     __syncthreads();
-    init_tile<NB>(P, S.wt, S.s_t, S.z_t, S.lo_t, S.hi_t, tg);
+    init_tile<NB>(P, S.wh, S.s_t, S.z_t, S.lo_t, S.hi_t, tg);
     __syncthreads();
-    run_rounds<NB, L, false, FULL>(P, S.wt, S.s_t, S.z_t, S.lo_t, S.hi_t, S.f_t, S.tab, S.list,
-                                   S.acc_w, tg, 0);
+    run_groups<NB, L, false, FULL, DIRECT>(P, S.wh, S.s_t, S.z_t, S.lo_t, S.hi_t, S.f_t, S.tab,
+                                           S.acc_w, S.thr, S.beta, t0, tg, 0);
     __syncthreads();
-    write_tile<NB>(P, S.wt, S.s_t, S.z_t, S.cbuf, t0, tg);
-    for (int i = threadIdx.x; i < tg; i += kThreads) {
-        P.fk[t0 + i] = S.f_t[i];
-        if (P.group_rounds) P.group_rounds[t0 + i] = K > 0 ? (uint8_t)(S.f_t[i] + 1) : 0;
-    }
+    if (!DIRECT) write_tile<NB>(P, S.wh, S.s_t, S.z_t, S.f_t, true, t0, tg);
+    // the largest f of the tile (for the fixup's staleness test)
+    int mf = 0;
+    for (int i = threadIdx.x; i < tg; i += kThreads) mf = max(mf, DIRECT ? (int)__ldcg(P.fk + t0 + i) : (int)S.f_t[i]);
+    atomicMax(&maxf, mf);
     // this tile's per-round sums (16-bit chunks) -> 128-bit global sums
     for (int i = threadIdx.x; i < 2 * K; i += kThreads) {
         unsigned __int128 v = 0;
@@ -628,42 +724,47 @@ __global__ void __launch_bounds__(kThreads) hqq_search_kernel(const __grid_const
             if (hi + carry) atomicAdd(P.acc + 2 * i + 1, hi + carry);
         }
     }
-    // the last tile to finish applies the stop rule once for the whole tensor
+    __syncthreads();
+    if (threadIdx.x == 0) P.tile_maxf[blockIdx.x] = (uint8_t)maxf;
+    // the last tile to finish applies the stop rule once for the whole tensor and lists the
+    // tiles that hold a group whose own last round lies past the kept round
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) last = atomicAdd(&ctl_of(P)->done, 1u) == gridDim.x - 1;
     __syncthreads();
-    if (last && threadIdx.x == 0) {
+    if (last) {
         __threadfence();
-        stop_rule(P);
+        if (threadIdx.x == 0) stop_rule(P);
+        __syncthreads();
+        Ctl *c = ctl_of(P);
+        const int b = *(volatile int *)&c->b;
+        for (int t = threadIdx.x; t < (int)gridDim.x; t += kThreads)
+            if ((int)__ldcg(P.tile_maxf + t) > b) P.stale[atomicAdd(&c->nstale, 1)] = t;
     }
 }
 
-// Recomputes the tiles that hold a group whose own last round lies past the kept round b.
-template <int NB, int L, bool FULL>
-__global__ void __launch_bounds__(kThreads) hqq_fixup_kernel(const __grid_constant__ QParams P,
-                                                              int64_t ntiles) {
+// Recomputes the stale tiles listed by the search kernel.
+template <int NB, int L, bool FULL, bool DIRECT>
+__global__ void __launch_bounds__(kThreads, 2) hqq_fixup_kernel(const __grid_constant__ QParams P) {
     extern __shared__ __align__(16) unsigned char smem[];
+    Ctl *c = ctl_of(P);
+    const int nstale = __ldcg(&c->nstale);
+    if ((int)blockIdx.x >= nstale) return;
     Smem<NB, L> S(smem, P);
-    const int b = __ldcg(&ctl_of(P)->b);
-    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-        const int64_t t0 = tile * P.tile;
+    const int b = __ldcg(&c->b);
+    load_constants(P, S);
+    for (int si = blockIdx.x; si < nstale; si += gridDim.x) {
+        const int64_t t0 = (int64_t)__ldcg(P.stale + si) * P.tile;
         const int tg = (int)min((int64_t)P.tile, P.G - t0);
-        int stale = 0;
-        for (int i = threadIdx.x; i < tg; i += kThreads) {
-            const uint8_t f = P.fk[t0 + i];
-            S.f_t[i] = f;
-            stale |= (int)f > b;
-        }
-        if (__syncthreads_or(stale) == 0) continue;
-        stage_tile(P, S.wt, t0, tg);
+        for (int i = threadIdx.x; i < tg; i += kThreads) S.f_t[i] = __ldcg(P.fk + t0 + i);
+        stage_tile(P, S.wh, t0, tg);
         __syncthreads();
-        init_tile<NB>(P, S.wt, S.s_t, S.z_t, S.lo_t, S.hi_t, tg);
+        init_tile<NB>(P, S.wh, S.s_t, S.z_t, S.lo_t, S.hi_t, tg);
         __syncthreads();
-        run_rounds<NB, L, true, FULL>(P, S.wt, S.s_t, S.z_t, S.lo_t, S.hi_t, S.f_t, S.tab, S.list,
-                                      nullptr, tg, b);
+        run_groups<NB, L, true, FULL, DIRECT>(P, S.wh, S.s_t, S.z_t, S.lo_t, S.hi_t, S.f_t, S.tab,
+                                              nullptr, S.thr, S.beta, t0, tg, b);
         __syncthreads();
-        write_tile<NB>(P, S.wt, S.s_t, S.z_t, S.cbuf, t0, tg);
+        if (!DIRECT) write_tile<NB>(P, S.wh, S.s_t, S.z_t, S.f_t, false, t0, tg);
         __syncthreads();
     }
 }
@@ -838,10 +939,10 @@ void launch_dequant(const uint8_t *pk, const __half *sc, const __half *ze, int64
 // ------------------------------------------------------------------------------------------
 struct Plan {
     int64_t N, G;
-    int g, P, L, stride, tile;
+    int g, P, L, stride, tile;  // stride: floats per tile row
     int64_t ntiles;
     bool aligned;  // packed words can be written per tile
-    size_t ws_acc, ws_fk, ws_codes, ws_total;
+    size_t ws_acc, ws_fk, ws_tile, ws_stale, ws_codes, ws_total;
 };
 
 int64_t gcd64(int64_t a, int64_t b) {
@@ -869,42 +970,52 @@ int make_plan(int64_t rows, int64_t cols, int nbits, int64_t group_size, int axi
     while (P < pl->g) P *= 2;
     pl->P = P;
     pl->L = P / kE;
-    pl->stride = P + 4;
-    const int budget = 16384;  // floats of tile rows per CTA (64 KB)
-    const int cap = (int)std::min<int64_t>(10240 / pl->g, budget / pl->stride);
-    const int cap2 = std::min(cap, kWarps * 64);  // each warp owns at most 64 groups
-    if (axis == 1) {
-        // tiles of a multiple of 320 elements: word (8, 16, 10 codes) and 16-byte aligned
-        const int unit = (int)(320 / gcd64(pl->g, 320));
-        pl->tile = unit * std::max(1, cap2 / unit);
-    } else {
-        pl->tile = 80 * std::max(1, cap2 / 80);  // columns; 80 = lcm(8, 16, 10)
+    pl->stride = P + (P >= 64 ? 8 : 0);  // halves per tile row (the padding staggers banks)
+    const int target = 40960;            // halves of W per tile
+    const int cap = std::max(1, target / pl->stride);
+    const int unit = axis == 1 ? (int)(320 / gcd64(pl->g, 320))  // tiles of 320k elements: word
+                               : 80;                             // (8, 16, 10 codes) and 16-byte
+    pl->tile = unit * std::max(1, cap / unit);                   // aligned; 80 = lcm(8, 16, 10)
+    // two CTAs per SM: keep the whole shared-memory layout within 110 KB
+    while (pl->tile > unit &&
+           smem_layout(pl->tile, pl->stride, 1 << nbits, pl->L, iters).total > 110 * 1024)
+        pl->tile -= unit;
+    // spread the groups evenly over whole waves of resident CTAs (two per SM)
+    {
+        const int64_t slots = 2 * 148;  // B200: 148 SMs
+        const int64_t want = (pl->G + pl->tile - 1) / pl->tile;
+        const int64_t waves = (want + slots - 1) / slots;
+        const int64_t per = (pl->G + waves * slots - 1) / (waves * slots);
+        const int64_t even = (per + unit - 1) / unit * unit;
+        if (even < pl->tile) pl->tile = (int)even;
     }
-    if (pl->tile > kWarps * 64) return HQQ_ERR_UNSUPPORTED;
     pl->ntiles = (pl->G + pl->tile - 1) / pl->tile;
     pl->aligned = axis == 1 || (pl->G % cpw_of(nbits) == 0);
     const int K = iters > 0 ? iters : 1;
-    pl->ws_acc = (size_t)4 * K * sizeof(u64) + 16;  // per-round sums + control words
+    pl->ws_acc = (size_t)4 * K * sizeof(u64) + 16;  // per-round sums + control words (zeroed)
     pl->ws_fk = (size_t)((pl->G + 15) / 16 * 16);
+    pl->ws_tile = (size_t)((pl->ntiles + 15) / 16 * 16);
+    pl->ws_stale = (size_t)(4 * pl->ntiles + 15) / 16 * 16;
     pl->ws_codes = pl->aligned ? 0 : (size_t)((N + 15) / 16 * 16);
-    pl->ws_total = pl->ws_acc + pl->ws_fk + pl->ws_codes;
+    pl->ws_total = pl->ws_acc + pl->ws_fk + pl->ws_tile + pl->ws_stale + pl->ws_codes;
     return HQQ_OK;
 }
 
 bool aligned_to(const void *p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
 
-template <int NB, int L, bool FULL>
+
+template <int NB, int L, bool FULL, bool DIRECT>
 cudaError_t launch_quant(const QParams &P, int64_t ntiles, cudaStream_t st) {
     const SmemLayout lay = smem_layout(P.tile, P.stride, 1 << NB, L, P.K);
-    cudaError_t e = cudaFuncSetAttribute(hqq_search_kernel<NB, L, FULL>,
+    cudaError_t e = cudaFuncSetAttribute(hqq_search_kernel<NB, L, FULL, DIRECT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(hqq_fixup_kernel<NB, L, FULL>,
+    e = cudaFuncSetAttribute(hqq_fixup_kernel<NB, L, FULL, DIRECT>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total);
     if (e != cudaSuccess) return e;
-    hqq_search_kernel<NB, L, FULL><<<(unsigned)ntiles, kThreads, lay.total, st>>>(P);
-    const unsigned fix_blocks = (unsigned)std::min<int64_t>(ntiles, 148 * 4);
-    hqq_fixup_kernel<NB, L, FULL><<<fix_blocks, kThreads, lay.total, st>>>(P, ntiles);
+    hqq_search_kernel<NB, L, FULL, DIRECT><<<(unsigned)ntiles, kThreads, lay.total, st>>>(P);
+    const unsigned fix_blocks = (unsigned)std::min<int64_t>(ntiles, 148 * 2);  // one wave
+    hqq_fixup_kernel<NB, L, FULL, DIRECT><<<fix_blocks, kThreads, lay.total, st>>>(P);
     if (P.codes_u8) {
         const int64_t nw = (P.N + Pack<NB>::cpw - 1) / Pack<NB>::cpw;
         const unsigned blocks = (unsigned)std::min<int64_t>((nw + 255) / 256, 148 * 16);
@@ -913,24 +1024,29 @@ cudaError_t launch_quant(const QParams &P, int64_t ntiles, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-template <int NB>
-cudaError_t launch_quant_l(const QParams &P, int L, bool full, int64_t ntiles, cudaStream_t st) {
-    if (full) {  // group size a power of two >= 16: every slot of a lane holds an element
-        switch (L) {
-        case 1: return launch_quant<NB, 1, true>(P, ntiles, st);
-        case 2: return launch_quant<NB, 2, true>(P, ntiles, st);
-        case 4: return launch_quant<NB, 4, true>(P, ntiles, st);
-        case 8: return launch_quant<NB, 8, true>(P, ntiles, st);
-        default: return launch_quant<NB, 16, true>(P, ntiles, st);
-        }
-    }
+template <int NB, bool FULL, bool DIRECT>
+cudaError_t launch_quant_l(const QParams &P, int L, int64_t ntiles, cudaStream_t st) {
     switch (L) {
-    case 1: return launch_quant<NB, 1, false>(P, ntiles, st);
-    case 2: return launch_quant<NB, 2, false>(P, ntiles, st);
-    case 4: return launch_quant<NB, 4, false>(P, ntiles, st);
-    case 8: return launch_quant<NB, 8, false>(P, ntiles, st);
-    default: return launch_quant<NB, 16, false>(P, ntiles, st);
+    case 1: return launch_quant<NB, 1, FULL, DIRECT>(P, ntiles, st);
+    case 2: return launch_quant<NB, 2, FULL, DIRECT>(P, ntiles, st);
+    case 4: return launch_quant<NB, 4, FULL, DIRECT>(P, ntiles, st);
+    case 8: return launch_quant<NB, 8, FULL, DIRECT>(P, ntiles, st);
+    default: return launch_quant<NB, 16, FULL, DIRECT>(P, ntiles, st);
     }
+}
+
+// full: group size a power of two >= 16 (every slot of a lane holds an element); direct:
+// axis 1 with 2- or 4-bit codes and group size a multiple of 16 (a lane's 16 codes are whole
+// bytes of the output)
+template <int NB>
+cudaError_t launch_quant_nb(const QParams &P, int L, bool full, bool direct, int64_t ntiles,
+                            cudaStream_t st) {
+    if (NB != 3 && direct) {
+        return full ? launch_quant_l<NB, true, NB != 3>(P, L, ntiles, st)
+                    : launch_quant_l<NB, false, NB != 3>(P, L, ntiles, st);
+    }
+    return full ? launch_quant_l<NB, true, false>(P, L, ntiles, st)
+                : launch_quant_l<NB, false, false>(P, L, ntiles, st);
 }
 
 }  // namespace
@@ -1004,8 +1120,11 @@ extern "C" int hqq_quantize(const void *W, int64_t rows, int64_t cols, int nbits
     P.s_out = s_f32;
     P.z_out = z_f32;
     P.acc = (u64 *)workspace;
-    P.fk = (uint8_t *)workspace + pl.ws_acc;
-    P.codes_u8 = pl.aligned ? nullptr : (uint8_t *)workspace + pl.ws_acc + pl.ws_fk;
+    uint8_t *wsp = (uint8_t *)workspace;
+    P.fk = wsp + pl.ws_acc;
+    P.tile_maxf = wsp + pl.ws_acc + pl.ws_fk;
+    P.stale = (int *)(wsp + pl.ws_acc + pl.ws_fk + pl.ws_tile);
+    P.codes_u8 = pl.aligned ? nullptr : wsp + pl.ws_acc + pl.ws_fk + pl.ws_tile + pl.ws_stale;
     P.iters_run = iters_run;
     P.err_trace = (u64 *)err_trace;
     P.group_rounds = group_rounds;
@@ -1022,11 +1141,12 @@ extern "C" int hqq_quantize(const void *W, int64_t rows, int64_t cols, int nbits
     }
     cudaStream_t st = (cudaStream_t)stream;
     if (cudaMemsetAsync(workspace, 0, pl.ws_acc, st) != cudaSuccess) return HQQ_ERR_CUDA;
+    const bool direct = axis == 1 && pl.g % 16 == 0;
     cudaError_t e;
     switch (nbits) {
-    case 4: e = launch_quant_l<4>(P, pl.L, pl.g == pl.P, pl.ntiles, st); break;
-    case 3: e = launch_quant_l<3>(P, pl.L, pl.g == pl.P, pl.ntiles, st); break;
-    default: e = launch_quant_l<2>(P, pl.L, pl.g == pl.P, pl.ntiles, st); break;
+    case 4: e = launch_quant_nb<4>(P, pl.L, pl.g == pl.P, direct, pl.ntiles, st); break;
+    case 3: e = launch_quant_nb<3>(P, pl.L, pl.g == pl.P, false, pl.ntiles, st); break;
+    default: e = launch_quant_nb<2>(P, pl.L, pl.g == pl.P, direct, pl.ntiles, st); break;
     }
     return e == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
 }

@@ -36,6 +36,28 @@ ISSUE_LANES_PER_SM = 128     # 4 SM sub-partitions x 32 lanes issue one instruct
 ALU_OPS_INIT, ALU_OPS_ROUND, ALU_OPS_FINAL = 3, 12, 6   # algorithmic ops per weight
 
 
+PROFILE = os.path.join(ROOT, "profiles", "hqq_search_kernel_4096x4096_b4g64.md")
+KERNEL_SRC = os.path.join(ROOT, "free_weight_quantization_b200", "csrc", "hqq_b200.cu")
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the search kernel from the committed ncu summary, or None
+    when the kernel source has changed since that capture."""
+    import hashlib
+    try:
+        text = open(PROFILE).read()
+        src = hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    fields = dict(l.split(":", 1) for l in text.splitlines() if l.startswith(("source-sha256:", "traffic-bytes-per-launch:")))
+    if fields.get("source-sha256", "").strip() != src:
+        return None
+    try:
+        return float(fields["traffic-bytes-per-launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def peaks():
     p = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "src": "fallback"}
     try:
@@ -167,7 +189,7 @@ def cpu_baseline():
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--steps", type=int, default=5000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -292,9 +314,9 @@ def main():
         if rounds is not None:
             alg_ops = N * (ALU_OPS_INIT + ALU_OPS_FINAL) + GROUP * rounds * ALU_OPS_ROUND
             ach = alg_ops / q_s / 1e12
-            roofline = {"bound": "alu", "kernel": "hqq_quantize (search + fixup kernels)",
+            roofline = {"bound": "alu", "kernel": "hqq_quantize (hqq_stream_kernel + hqq_stream_fixup_kernel)",
                         "achieved": ach, "peak": alu_peak, "unit": "Tops/s", "frac": ach / alu_peak,
-                        "traffic": None,
+                        "traffic": profiled_traffic(),
                         "peak_src": f"148 SMs x 128 lanes x {pk['sm_max_mhz']:.0f} MHz (max clock)",
                         "alg_ops_per_launch": alg_ops, "group_rounds": rounds}
         line = {

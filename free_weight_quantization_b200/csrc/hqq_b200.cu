@@ -635,10 +635,12 @@ struct Smem {
 // workspace words after the per-round sums: tiles finished, kept round, rounds measured,
 // number of stale tiles; then the per-tile largest f and the list of stale tiles
 struct Ctl {
-    unsigned done;
-    int b;
-    int run;
-    int nstale;
+    unsigned done;      // tiles (or warps, streaming engine) finished
+    int b;              // kept round
+    int run;            // rounds whose MAE was computed
+    int nstale;         // stale tiles (tile engine)
+    unsigned long long work;  // next group to hand out (streaming engine)
+    unsigned long long pad;
 };
 
 __device__ __forceinline__ Ctl *ctl_of(const QParams &P) {
@@ -766,6 +768,476 @@ __global__ void __launch_bounds__(kThreads, 2) hqq_fixup_kernel(const __grid_con
         __syncthreads();
         if (!DIRECT) write_tile<NB>(P, S.wh, S.s_t, S.z_t, S.f_t, false, t0, tg);
         __syncthreads();
+    }
+}
+
+// ==========================================================================================
+// Streaming engine (axis 1): one lane per group
+//
+// Each lane holds one whole group: its fp16 row in registers (P/2 words), its own table of the
+// 2^b reconstructions in a private shared-memory column, and its running state.  Lanes take
+// groups from a global counter (one atomic per warp and refill), so the work stays balanced
+// to the end, and each lane copies its next group's row into a shared-memory slot with
+// cp.async one group ahead.  The pairwise group sums are an 8-element tree per chunk and a
+// compile-time stack over the chunks; no shuffles are needed.
+// ==========================================================================================
+template <int P>
+struct SRow {
+    uint32_t h[P / 2];  // fp16 pairs: element 2i in the low half
+};
+
+__device__ __forceinline__ float half_lo(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v & 0xffffu))); }
+__device__ __forceinline__ float half_hi(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v >> 16))); }
+
+// push a chunk's sum onto a pairwise stack: after chunk ch, level l holds the sum of the last
+// 2^l chunks whenever bit l of ch + 1 is set; the final entry is the whole pairwise sum
+template <int LOGN>
+__device__ __forceinline__ void pw_push(float (&stk)[LOGN + 1], int ch, float v) {
+#pragma unroll
+    for (int lvl = 0; lvl <= LOGN; ++lvl) {
+        if ((ch >> lvl) & 1) {
+            v = __fadd_rn(stk[lvl], v);
+        } else {
+            stk[lvl] = v;
+            return;
+        }
+    }
+}
+
+__device__ __forceinline__ float tree8(const float *x) {
+    return __fadd_rn(__fadd_rn(__fadd_rn(x[0], x[1]), __fadd_rn(x[2], x[3])),
+                     __fadd_rn(__fadd_rn(x[4], x[5]), __fadd_rn(x[6], x[7])));
+}
+
+// One proximal round over a lane's group [HQQ 算法解读, "第二拍"] with e = 0 for every element.
+// Returns the group's error sum, the zero-update sum (z_new times g), the largest residual
+// and (DIRECT) the round's codes.
+template <int NB, int P, bool DIRECT>
+struct SCodes {  // a lane's codes of the current round, in the output's packed format
+    static constexpr int kWords = DIRECT ? P * NB / 32 : 1;
+    uint32_t w[kWords];
+};
+
+template <int NB, int P, bool FULL, bool CLIP, bool DIRECT>
+__device__ __forceinline__ void stream_round(const SRow<P> &row, int g, float s, float z,
+                                             uint32_t tab_adj, float &esum, float &zsum,
+                                             float &maxr, SCodes<NB, P, DIRECT> &codes) {
+    constexpr int NCH = P / 8;
+    constexpr int LOGN = NCH == 1 ? 0 : NCH == 2 ? 1 : NCH == 4 ? 2 : NCH == 8 ? 3 : NCH == 16 ? 4 : 5;
+    constexpr float kQmax = (float)((1 << NB) - 1);
+    float sa[LOGN + 1], st[LOGN + 1];
+    maxr = 0.0f;
+#pragma unroll
+    for (int ch = 0; ch < NCH; ++ch) {
+        float ar[8], tm[8];
+#pragma unroll
+        for (int m2 = 0; m2 < 8; m2 += 2) {
+            const float2 wp = __half22float2(*reinterpret_cast<const __half2 *>(&row.h[(8 * ch + m2) / 2]));
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int m = m2 + h, j = 8 * ch + m;
+                const float w = h ? wp.y : wp.x;
+                const float ws = __fmul_rn(w, s);
+                float t = __fadd_rn(ws, z);
+                if (CLIP) t = fminf(fmaxf(t, 0.0f), kQmax);
+                const float u = __fadd_rn(t, kMagic);
+                const float qf = __fsub_rn(u, kMagic);
+                const uint32_t bits = __float_as_uint(u);
+                float what;
+                asm volatile("ld.shared.f32 %0, [%1];" : "=f"(what) : "r"(tab_adj + (bits << 7)));
+                if (DIRECT) {  // code j at bit NB*j of the group's words (low NB bits of `bits`)
+                    constexpr int CPW = 32 / NB;
+                    uint32_t d;
+                    asm("bfi.b32 %0, %1, %2, %3, %4;" : "=r"(d)
+                        : "r"(bits), "r"(j % CPW == 0 ? 0u : codes.w[j / CPW]), "r"(NB * (j % CPW)), "r"(NB));
+                    codes.w[j / CPW] = d;
+                }
+                const bool valid = FULL || (j < g);
+                const float a = fabsf(__fsub_rn(w, what));
+                ar[m] = valid ? a : 0.0f;
+                tm[m] = valid ? __fsub_rn(qf, ws) : 0.0f;  // q - (W - 0)*s
+                maxr = fmaxf(maxr, ar[m]);
+            }
+        }
+        pw_push<LOGN>(sa, ch, tree8(ar));
+        pw_push<LOGN>(st, ch, tree8(tm));
+    }
+    esum = sa[LOGN];
+    zsum = st[LOGN];
+}
+
+// The rare paths read the group's row back from global memory (it is cached), so the
+// unrolled register copy stays out of them.
+//
+// The zero-update sum with the exact lp shrink e = shrink(W - W_hat) for every element:
+// pairwise in the same order as stream_round (8-element chunks, then a stack over chunks).
+template <int NB>
+__device__ __noinline__ float group_zsum_shrink(const __half *wrow, int g, int P, float s,
+                                                float z, uint32_t tab_adj, double beta,
+                                                double p) {
+    constexpr float kQmax = (float)((1 << NB) - 1);
+    float stk[6];
+    const int nch = P / 8;
+    for (int ch = 0; ch < nch; ++ch) {
+        float tm[8];
+        for (int m = 0; m < 8; ++m) {
+            const int j = 8 * ch + m;
+            float term = 0.0f;
+            if (j < g) {
+                const float w = __half2float(wrow[j]);
+                const float t = fminf(fmaxf(__fadd_rn(__fmul_rn(w, s), z), 0.0f), kQmax);
+                const float u = __fadd_rn(t, kMagic);
+                const float qf = __fsub_rn(u, kMagic);
+                float what;
+                asm volatile("ld.shared.f32 %0, [%1];" : "=f"(what) : "r"(tab_adj + (__float_as_uint(u) << 7)));
+                const float e = shrink_lp(__fsub_rn(w, what), beta, p);
+                term = __fsub_rn(qf, __fmul_rn(__fsub_rn(w, e), s));
+            }
+            tm[m] = term;
+        }
+        float v = tree8(tm);
+        int lvl = 0;
+        for (; (ch >> lvl) & 1; ++lvl) v = __fadd_rn(stk[lvl], v);
+        stk[lvl] = v;
+    }
+    int top = 0;
+    while ((1 << top) < nch) ++top;
+    return stk[top];
+}
+
+// final codes of a lane's group with the kept zero, written to the packed output
+// [HQQ 算法解读, "第二拍" and "为什么一定要分组"].  DIRECT: the group covers whole 32-bit words
+// of the output, stored as they are.
+template <int NB, int P>
+__device__ __forceinline__ void group_store_codes(const QParams &Pm, const SRow<P> &row,
+                                                  int64_t grp, float s, float z) {
+    constexpr int CPW = 32 / NB;  // NB in {2, 4}; g = P and P*NB % 32 == 0
+    constexpr float kQmax = (float)((1 << NB) - 1);
+    uint32_t *dst = reinterpret_cast<uint32_t *>(Pm.packed) + grp * (P / CPW);
+#pragma unroll
+    for (int wi = 0; wi < P / CPW; ++wi) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int c = 0; c < CPW; ++c) {
+            const int j = wi * CPW + c;
+            const float w = (j & 1) ? half_hi(row.h[j / 2]) : half_lo(row.h[j / 2]);
+            const float t = fminf(fmaxf(__fadd_rn(__fmul_rn(w, s), z), 0.0f), kQmax);
+            word |= (__float_as_uint(__fadd_rn(t, kMagic)) & ((1u << NB) - 1u)) << (NB * c);
+        }
+        dst[wi] = word;
+    }
+}
+
+// Otherwise the codes are OR-ed into the zeroed output one 32-bit word at a time (a word may
+// be shared with the neighbouring group); clear = true first clears the group's own bits.
+template <int NB>
+__device__ __noinline__ void group_or_codes(const QParams &Pm, const __half *wrow, int64_t grp,
+                                            float s, float z, bool clear) {
+    constexpr int CPW = NB == 4 ? 8 : NB == 2 ? 16 : 10;  // codes per 32-bit word
+    constexpr uint32_t MASK = (1u << NB) - 1u;
+    constexpr float kQmax = (float)((1 << NB) - 1);
+    const int g = Pm.g;
+    const int64_t n0 = grp * g;
+    int64_t wi = n0 / CPW;
+    int c = (int)(n0 - wi * CPW);
+    uint32_t word = 0, mask = 0;
+    uint32_t *out = reinterpret_cast<uint32_t *>(Pm.packed);
+    for (int j = 0; j < g; ++j) {
+        const float t = fminf(fmaxf(__fadd_rn(__fmul_rn(__half2float(wrow[j]), s), z), 0.0f), kQmax);
+        word |= (__float_as_uint(__fadd_rn(t, kMagic)) & MASK) << (NB * c);
+        mask |= MASK << (NB * c);
+        if (++c == CPW || j == g - 1) {  // the packed size is a whole number of words here
+            if (clear) atomicAnd(out + wi, ~mask);
+            atomicOr(out + wi, word);
+            ++wi;
+            c = 0;
+            word = 0;
+            mask = 0;
+        }
+    }
+}
+
+template <int NB, int P, bool FULL>
+__device__ __forceinline__ void group_init(const SRow<P> &row, int g, float eps, float smax,
+                                           float &s, float &z, float &lo, float &hi) {
+    constexpr float kQmax = (float)((1 << NB) - 1);
+    // min and max in fp16 pairs (exact); padded slots repeat element 0
+    __half2 mn2 = *reinterpret_cast<const __half2 *>(&row.h[0]), mx2 = mn2;
+#pragma unroll
+    for (int i = 1; i < P / 2; ++i) {
+        const __half2 v = *reinterpret_cast<const __half2 *>(&row.h[i]);
+        mn2 = __hmin2(mn2, v);
+        mx2 = __hmax2(mx2, v);
+    }
+    const float mn = fminf(__low2float(mn2), __high2float(mn2));
+    const float mx = fmaxf(__low2float(mx2), __high2float(mx2));
+    // [HQQ 算法解读, "第一拍：min-max 给一个可用的初值"]
+    const float d = __fsub_rn(mx, mn);
+    s = (d < eps) ? 1.0f : __fdiv_rn(kQmax, d);
+    s = fminf(s, smax);
+    z = __fsub_rn(0.0f, __fmul_rn(mn, s));
+    lo = __fmul_rn(mn, s);
+    hi = __fmul_rn(mx, s);
+}
+
+// row of group `grp` into registers; slots past g repeat element 0 (inside the group's range)
+template <int P, bool FULL, bool ALIGN16>
+__device__ __forceinline__ void load_row(SRow<P> &row, const __half *W, int64_t grp, int g,
+                                         const __half *slot) {
+    if (ALIGN16) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(slot);
+#pragma unroll
+        for (int v = 0; v < P / 8; ++v) {
+            if (FULL || 8 * v < g) {
+                const uint4 x = src[v];
+                row.h[4 * v] = x.x; row.h[4 * v + 1] = x.y; row.h[4 * v + 2] = x.z; row.h[4 * v + 3] = x.w;
+            }
+        }
+    } else {
+        const unsigned short *src = reinterpret_cast<const unsigned short *>(W + grp * g);
+#pragma unroll
+        for (int j = 0; j < P; j += 2) {
+            const uint32_t a = (FULL || j < g) ? src[j] : 0u;
+            const uint32_t b = (FULL || j + 1 < g) ? src[j + 1] : 0u;
+            row.h[j / 2] = a | (b << 16);
+        }
+    }
+    if (!FULL) {
+        const uint32_t e0 = row.h[0] & 0xffffu;
+#pragma unroll
+        for (int j = 0; j < P; ++j)
+            if (j >= g) row.h[j / 2] = (j & 1) ? ((row.h[j / 2] & 0xffffu) | (e0 << 16)) : ((row.h[j / 2] & 0xffff0000u) | e0);
+    }
+}
+
+template <int P, bool ALIGN16>
+__device__ __forceinline__ void prefetch_row(__half *slot, const __half *W, int64_t grp, int g) {
+    if (ALIGN16) {
+        const char *src = reinterpret_cast<const char *>(W + grp * g);
+        const uint32_t dst = (uint32_t)__cvta_generic_to_shared(slot);
+#pragma unroll
+        for (int v = 0; v < P / 8; ++v)
+            if (8 * v < g)
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + 16 * v), "l"(src + 16 * v));
+        asm volatile("cp.async.commit_group;" ::);
+    }
+}
+
+__device__ __forceinline__ void prefetch_wait() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+struct StreamSmem {
+    static __host__ __device__ int bytes(int P, int nq, int K) {
+        const int Kc = K > 0 ? K : 1;
+        return kWarps * (nq * 32 * 4)                 // tables: [NQ][32] floats per warp
+               + kWarps * 2 * Kc * 4 * 4              // per-warp round counters
+               + kWarps * 32 * P * 2                  // prefetch slots: one row per lane
+               + ((Kc * 4 + 15) / 16 * 16) + Kc * 8;  // thresholds and betas
+    }
+};
+
+// claim one group per requesting lane from the global counter (one atomic per warp)
+__device__ __forceinline__ int64_t claim(const QParams &Pm, bool want) {
+    const unsigned lane = threadIdx.x & 31;
+    const unsigned m = __ballot_sync(kFull, want);
+    unsigned long long base = 0;
+    if (lane == 0 && m) base = atomicAdd(&ctl_of(Pm)->work, (unsigned long long)__popc(m));
+    base = __shfl_sync(kFull, base, 0);
+    const int64_t id = (int64_t)base + __popc(m & ((1u << lane) - 1u));
+    return (want && id < Pm.G) ? id : -1;
+}
+
+template <int NB, int P, bool FULL, bool ALIGN16, bool DIRECT>
+__global__ void __launch_bounds__(kThreads) hqq_stream_kernel(const __grid_constant__ QParams Pm) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    constexpr int NQ = 1 << NB;
+    constexpr float kQmax = (float)(NQ - 1);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int K = Pm.K, g = Pm.g;
+    const int Kc = K > 0 ? K : 1;
+    float *tabw = reinterpret_cast<float *>(smem) + warp * NQ * 32;
+    unsigned *acc = reinterpret_cast<unsigned *>(smem + kWarps * NQ * 32 * 4);
+    unsigned *acc_w = acc + warp * 8 * Kc;
+    __half *slot = reinterpret_cast<__half *>(smem + kWarps * NQ * 32 * 4 + kWarps * 8 * Kc * 4) +
+                   (warp * 32 + lane) * P;
+    float *thr_s = reinterpret_cast<float *>(smem + kWarps * NQ * 32 * 4 + kWarps * 8 * Kc * 4 +
+                                             kWarps * 32 * P * 2);
+    double *beta_s = reinterpret_cast<double *>(reinterpret_cast<unsigned char *>(thr_s) +
+                                                (Kc * 4 + 15) / 16 * 16);
+    __shared__ bool last;
+    for (int i = threadIdx.x; i < kWarps * 8 * Kc; i += kThreads) acc[i] = 0;
+    for (int i = threadIdx.x; i < K; i += kThreads) { thr_s[i] = Pm.thr[i]; beta_s[i] = Pm.beta[i]; }
+    __syncthreads();
+    const float thr_last = K > 0 ? thr_s[K - 1] : 0.0f;
+    const float inv_g = 1.0f / (float)g;  // exact for FULL (g = 2^k)
+    const uint32_t tab_adj = (uint32_t)__cvta_generic_to_shared(tabw + lane) - (0x4B400000u << 7);
+
+    SRow<P> row;
+#pragma unroll
+    for (int i = 0; i < P / 2; ++i) row.h[i] = 0;
+    SCodes<NB, P, DIRECT> codes;
+#pragma unroll
+    for (int i = 0; i < SCodes<NB, P, DIRECT>::kWords; ++i) codes.w[i] = 0;
+    float s = 1.0f, z = 0.0f, lo = 0.0f, hi = 0.0f;
+    int it = 0;
+    int64_t cur = -1;
+    int64_t nxt = claim(Pm, true);
+    if (nxt >= 0) prefetch_row<P, ALIGN16>(slot, Pm.W, nxt, g);
+    while (true) {
+        // ---- a lane without a group takes the prefetched one and prefetches another
+        const bool need = cur < 0 && nxt >= 0;
+        if (__any_sync(kFull, need)) {
+            if (need) {
+                prefetch_wait();
+                cur = nxt;
+                load_row<P, FULL, ALIGN16>(row, Pm.W, cur, g, slot);
+                group_init<NB, P, FULL>(row, g, Pm.eps_tiny, Pm.scale_max, s, z, lo, hi);
+                it = 0;
+            }
+            const int64_t n2 = claim(Pm, need);
+            if (need) {
+                nxt = n2;
+                if (nxt >= 0) prefetch_row<P, ALIGN16>(slot, Pm.W, nxt, g);
+            }
+        }
+        const bool active = cur >= 0;
+        if (!__any_sync(kFull, active)) break;
+        bool done = active && K == 0;
+        if (__any_sync(kFull, active && K > 0)) {
+            const int ri = min(it, max(K - 1, 0));
+            // the reconstructions W_hat = (k - z)/s of every code k, in this lane's column
+#pragma unroll
+            for (int k = 0; k < NQ; ++k) tabw[k * 32 + lane] = __fdiv_rn(__fsub_rn((float)k, z), s);
+            // no clip is needed when [lo + z, hi + z] rounds inside [0, 2^b - 1]; lanes without
+            // a group hold a zero row and zero state
+            const bool inside = __fadd_rn(lo, z) >= -0.5f && __fadd_rn(hi, z) < kQmax + 0.5f;
+            float esum, zsum, maxr;
+            if (__all_sync(kFull, inside))
+                stream_round<NB, P, FULL, false, DIRECT>(row, g, s, z, tab_adj, esum, zsum, maxr, codes);
+            else
+                stream_round<NB, P, FULL, true, DIRECT>(row, g, s, z, tab_adj, esum, zsum, maxr, codes);
+            // lp shrink: a residual above the round's safe threshold -> exact binary64 path
+            const bool slow = active && maxr > thr_s[ri];
+            if (slow) zsum = group_zsum_shrink<NB>(Pm.W + cur * g, g, P, s, z, tab_adj, beta_s[ri], Pm.p);
+            const float znew = FULL ? __fmul_rn(zsum, inv_g) : __fdiv_rn(zsum, (float)g);
+            if (active && K > 0) {
+                const bool frozen = !slow && !(maxr > thr_last) && (znew == z);
+                done = frozen || it == K - 1;
+                const u64 fx = err_fixed(esum);
+                add_fixed(acc_w + 4 * it, fx);
+                if (done && it + 1 < K) add_fixed(acc_w + 4 * (K + it + 1), fx);
+                if (!done) {
+                    z = znew;
+                    ++it;
+                }
+            }
+        }
+        if (done) {
+            // the codes of a group's last round are its final codes (z is the kept zero);
+            // with no round at all they are computed here
+            if constexpr (DIRECT) {
+                if (K == 0) {
+                    group_store_codes<NB, P>(Pm, row, cur, s, z);
+                } else {
+                    uint32_t *dst = reinterpret_cast<uint32_t *>(Pm.packed) + cur * (P * NB / 32);
+#pragma unroll
+                    for (int i = 0; i < SCodes<NB, P, DIRECT>::kWords; ++i) dst[i] = codes.w[i];
+                }
+            } else {
+                group_or_codes<NB>(Pm, Pm.W + cur * g, cur, s, z, false);
+            }
+            write_meta(Pm, cur, s, z, it);
+            cur = -1;
+            // an idle lane holds a zero row and zero state, inside every range
+#pragma unroll
+            for (int i = 0; i < P / 2; ++i) row.h[i] = 0;
+            s = 1.0f; z = 0.0f; lo = 0.0f; hi = 0.0f;
+        }
+    }
+    // this warp's per-round sums (16-bit chunks) -> 128-bit global sums
+    __syncwarp();
+    for (int i = lane; i < 2 * K; i += 32) {
+        const unsigned *c = acc_w + 4 * i;
+        const unsigned __int128 v = (unsigned __int128)c[0] + ((unsigned __int128)c[1] << 16) +
+                                    ((unsigned __int128)c[2] << 32) + ((unsigned __int128)c[3] << 48);
+        const u64 lo64 = (u64)v, hi64 = (u64)(v >> 64);
+        if (lo64 | hi64) {
+            const u64 old = atomicAdd(Pm.acc + 2 * i, lo64);
+            const u64 carry = (old + lo64 < old) ? 1ull : 0ull;
+            if (hi64 + carry) atomicAdd(Pm.acc + 2 * i + 1, hi64 + carry);
+        }
+    }
+    // the last CTA to finish applies the stop rule once for the whole tensor
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) last = atomicAdd(&ctl_of(Pm)->done, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (last && threadIdx.x == 0) {
+        __threadfence();
+        stop_rule(Pm);
+    }
+}
+
+// Groups whose own last round f lies past the kept round b make exactly min(b, f) zero
+// updates again and rewrite their codes and metadata.  Nothing to do when b = iters - 1.
+template <int NB, int P, bool FULL, bool ALIGN16, bool DIRECT>
+__global__ void __launch_bounds__(kThreads) hqq_stream_fixup_kernel(const __grid_constant__ QParams Pm) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    constexpr int NQ = 1 << NB;
+    const int K = Pm.K, g = Pm.g;
+    const int b = __ldcg(&ctl_of(Pm)->b);
+    if (K == 0 || b >= K - 1) return;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float *tabw = reinterpret_cast<float *>(smem) + warp * NQ * 32;
+    const uint32_t tab_adj = (uint32_t)__cvta_generic_to_shared(tabw + lane) - (0x4B400000u << 7);
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t base = (int64_t)blockIdx.x * blockDim.x; base < Pm.G; base += stride) {
+        const int64_t grp = base + threadIdx.x;
+        const int f = grp < Pm.G ? (int)__ldcg(Pm.fk + grp) : 0;
+        const bool stale = grp < Pm.G && f > b;
+        if (!__any_sync(kFull, stale)) continue;
+        SRow<P> row;
+#pragma unroll
+        for (int i = 0; i < P / 2; ++i) row.h[i] = 0;
+        float s = 1.0f, z = 0.0f, lo = 0.0f, hi = 0.0f;
+        if (stale) {
+            if (ALIGN16) {  // synchronous load of the row
+                const uint4 *src = reinterpret_cast<const uint4 *>(Pm.W + grp * g);
+#pragma unroll
+                for (int v = 0; v < P / 8; ++v) {
+                    if (FULL || 8 * v < g) {
+                        const uint4 x = src[v];
+                        row.h[4 * v] = x.x; row.h[4 * v + 1] = x.y; row.h[4 * v + 2] = x.z; row.h[4 * v + 3] = x.w;
+                    }
+                }
+                if (!FULL) {
+                    const uint32_t e0 = row.h[0] & 0xffffu;
+#pragma unroll
+                    for (int j = 0; j < P; ++j)
+                        if (j >= g) row.h[j / 2] = (j & 1) ? ((row.h[j / 2] & 0xffffu) | (e0 << 16)) : ((row.h[j / 2] & 0xffff0000u) | e0);
+                }
+            } else {
+                load_row<P, FULL, false>(row, Pm.W, grp, g, nullptr);
+            }
+            group_init<NB, P, FULL>(row, g, Pm.eps_tiny, Pm.scale_max, s, z, lo, hi);
+        }
+        const int n = stale ? min(b, f) : 0;
+        for (int r = 0; __any_sync(kFull, r < n); ++r) {
+#pragma unroll
+            for (int k = 0; k < NQ; ++k) tabw[k * 32 + lane] = __fdiv_rn(__fsub_rn((float)k, z), s);
+            float esum, zsum, maxr;
+            SCodes<NB, P, false> nocodes;
+            stream_round<NB, P, FULL, true, false>(row, g, s, z, tab_adj, esum, zsum, maxr, nocodes);
+            const int rr = min(r, K - 1);
+            const bool slow = r < n && maxr > Pm.thr[rr];
+            if (slow) zsum = group_zsum_shrink<NB>(Pm.W + grp * g, g, P, s, z, tab_adj, Pm.beta[rr], Pm.p);
+            const float znew = FULL ? __fmul_rn(zsum, 1.0f / (float)g) : __fdiv_rn(zsum, (float)g);
+            if (r < n) z = znew;
+        }
+        if (stale) {
+            if constexpr (DIRECT) group_store_codes<NB, P>(Pm, row, grp, s, z);
+            else group_or_codes<NB>(Pm, Pm.W + grp * g, grp, s, z, true);
+            write_meta(Pm, grp, s, z, -1);
+        }
     }
 }
 
@@ -942,6 +1414,7 @@ struct Plan {
     int g, P, L, stride, tile;  // stride: floats per tile row
     int64_t ntiles;
     bool aligned;  // packed words can be written per tile
+    bool stream;   // axis 1 with groups up to 128 and a whole number of packed words
     size_t ws_acc, ws_fk, ws_tile, ws_stale, ws_codes, ws_total;
 };
 
@@ -991,8 +1464,11 @@ int make_plan(int64_t rows, int64_t cols, int nbits, int64_t group_size, int axi
     }
     pl->ntiles = (pl->G + pl->tile - 1) / pl->tile;
     pl->aligned = axis == 1 || (pl->G % cpw_of(nbits) == 0);
+    // the streaming engine: axis 1, 2- and 4-bit codes, groups of 16 .. 128 that are whole
+    // 32-bit words of the output (its codes are stored straight from registers)
+    pl->stream = axis == 1 && nbits != 3 && P <= 128 && pl->g == P && (pl->g * nbits) % 32 == 0;
     const int K = iters > 0 ? iters : 1;
-    pl->ws_acc = (size_t)4 * K * sizeof(u64) + 16;  // per-round sums + control words (zeroed)
+    pl->ws_acc = (size_t)4 * K * sizeof(u64) + 32;  // per-round sums + control words (zeroed)
     pl->ws_fk = (size_t)((pl->G + 15) / 16 * 16);
     pl->ws_tile = (size_t)((pl->ntiles + 15) / 16 * 16);
     pl->ws_stale = (size_t)(4 * pl->ntiles + 15) / 16 * 16;
@@ -1035,16 +1511,52 @@ cudaError_t launch_quant_l(const QParams &P, int L, int64_t ntiles, cudaStream_t
     }
 }
 
+template <int NB, int P, bool FULL, bool ALIGN16, bool DIRECT>
+cudaError_t launch_stream(const QParams &Pm, cudaStream_t st) {
+    const int smem = StreamSmem::bytes(P, 1 << NB, Pm.K);
+    auto k1 = hqq_stream_kernel<NB, P, FULL, ALIGN16, DIRECT>;
+    auto k2 = hqq_stream_fixup_kernel<NB, P, FULL, ALIGN16, DIRECT>;
+    cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148, per_sm = 1;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k1, kThreads, smem) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    const int64_t lanes_needed = (Pm.G + 31) / 32 * 32;
+    const unsigned blocks = (unsigned)std::max<int64_t>(
+        1, std::min<int64_t>((int64_t)sms * per_sm, (lanes_needed + kThreads - 1) / kThreads));
+    if (!DIRECT && cudaMemsetAsync(Pm.packed, 0, Pm.packed_bytes, st) != cudaSuccess)
+        return cudaGetLastError();
+    k1<<<blocks, kThreads, smem, st>>>(Pm);
+    const unsigned fix_blocks = (unsigned)std::min<int64_t>((int64_t)sms * per_sm,
+                                                            (Pm.G + kThreads - 1) / kThreads);
+    k2<<<std::max(1u, fix_blocks), kThreads, smem, st>>>(Pm);
+    return cudaGetLastError();
+}
+
+template <int NB>
+cudaError_t launch_stream_nb(const QParams &Pm, int P, cudaStream_t st) {
+    switch (P) {
+    case 16: return launch_stream<NB, 16, true, true, true>(Pm, st);
+    case 32: return launch_stream<NB, 32, true, true, true>(Pm, st);
+    case 64: return launch_stream<NB, 64, true, true, true>(Pm, st);
+    default: return launch_stream<NB, 128, true, true, true>(Pm, st);
+    }
+}
+
 // full: group size a power of two >= 16 (every slot of a lane holds an element); direct:
 // axis 1 with 2- or 4-bit codes and group size a multiple of 16 (a lane's 16 codes are whole
 // bytes of the output)
 template <int NB>
 cudaError_t launch_quant_nb(const QParams &P, int L, bool full, bool direct, int64_t ntiles,
                             cudaStream_t st) {
-    if (NB != 3 && direct) {
-        return full ? launch_quant_l<NB, true, NB != 3>(P, L, ntiles, st)
-                    : launch_quant_l<NB, false, NB != 3>(P, L, ntiles, st);
-    }
+    if (NB != 3 && direct && L == 16)
+        return full ? launch_quant<NB, 16, true, NB != 3>(P, ntiles, st)
+                    : launch_quant<NB, 16, false, NB != 3>(P, ntiles, st);
     return full ? launch_quant_l<NB, true, false>(P, L, ntiles, st)
                 : launch_quant_l<NB, false, false>(P, L, ntiles, st);
 }
@@ -1141,12 +1653,16 @@ extern "C" int hqq_quantize(const void *W, int64_t rows, int64_t cols, int nbits
     }
     cudaStream_t st = (cudaStream_t)stream;
     if (cudaMemsetAsync(workspace, 0, pl.ws_acc, st) != cudaSuccess) return HQQ_ERR_CUDA;
-    const bool direct = axis == 1 && pl.g % 16 == 0;
     cudaError_t e;
-    switch (nbits) {
-    case 4: e = launch_quant_nb<4>(P, pl.L, pl.g == pl.P, direct, pl.ntiles, st); break;
-    case 3: e = launch_quant_nb<3>(P, pl.L, pl.g == pl.P, false, pl.ntiles, st); break;
-    default: e = launch_quant_nb<2>(P, pl.L, pl.g == pl.P, direct, pl.ntiles, st); break;
+    if (pl.stream) {  // one lane per group
+        e = nbits == 4 ? launch_stream_nb<4>(P, pl.P, st) : launch_stream_nb<2>(P, pl.P, st);
+    } else {
+        const bool direct = axis == 1 && pl.g % 16 == 0;
+        switch (nbits) {
+        case 4: e = launch_quant_nb<4>(P, pl.L, pl.g == pl.P, direct, pl.ntiles, st); break;
+        case 3: e = launch_quant_nb<3>(P, pl.L, pl.g == pl.P, false, pl.ntiles, st); break;
+        default: e = launch_quant_nb<2>(P, pl.L, pl.g == pl.P, direct, pl.ntiles, st); break;
+        }
     }
     return e == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
 }

@@ -36,7 +36,7 @@ ISSUE_LANES_PER_SM = 128     # 4 SM sub-partitions x 32 lanes issue one instruct
 ALU_OPS_INIT, ALU_OPS_ROUND, ALU_OPS_FINAL = 3, 12, 6   # algorithmic ops per weight
 
 
-PROFILE = os.path.join(ROOT, "profiles", "hqq_search_kernel_4096x4096_b4g64.md")
+PROFILE = os.path.join(ROOT, "profiles", "hqq_stream_kernel_4096x4096_b4g64.md")
 KERNEL_SRC = os.path.join(ROOT, "free_weight_quantization_b200", "csrc", "hqq_b200.cu")
 
 

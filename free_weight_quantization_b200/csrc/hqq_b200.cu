@@ -113,20 +113,6 @@ __device__ __forceinline__ float seg_sum(float v) {
     return v;
 }
 
-template <int L>
-__device__ __forceinline__ float seg_max(float v) {
-#pragma unroll
-    for (int off = 1; off < L; off <<= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, off));
-    return v;
-}
-
-template <int L>
-__device__ __forceinline__ float seg_min(float v) {
-#pragma unroll
-    for (int off = 1; off < L; off <<= 1) v = fminf(v, __shfl_xor_sync(kFull, v, off));
-    return v;
-}
-
 template <int NB>
 struct Pack;  // codes per 32-bit output word
 template <> struct Pack<4> { static constexpr int cpw = 8; };
@@ -809,17 +795,17 @@ __device__ __forceinline__ float tree8(const float *x) {
                      __fadd_rn(__fadd_rn(x[4], x[5]), __fadd_rn(x[6], x[7])));
 }
 
-// One proximal round over a lane's group [HQQ 算法解读, "第二拍"] with e = 0 for every element.
-// Returns the group's error sum, the zero-update sum (z_new times g), the largest residual
-// and (DIRECT) the round's codes.
 template <int NB, int P, bool DIRECT>
 struct SCodes {  // a lane's codes of the current round, in the output's packed format
     static constexpr int kWords = DIRECT ? P * NB / 32 : 1;
     uint32_t w[kWords];
 };
 
-template <int NB, int P, bool FULL, bool CLIP, bool DIRECT>
-__device__ __forceinline__ void stream_round(const SRow<P> &row, int g, float s, float z,
+// One proximal round over a lane's group [HQQ 算法解读, "第二拍"] with e = 0 for every element.
+// Returns the group's error sum, the zero-update sum (z_new times g), the largest residual
+// and (DIRECT) the round's codes.  CLIP: clamp W*s + z to [0, 2^b - 1] before rounding.
+template <int NB, int P, bool CLIP, bool DIRECT>
+__device__ __forceinline__ void stream_round(const SRow<P> &row, float s, float z,
                                              uint32_t tab_adj, float &esum, float &zsum,
                                              float &maxr, SCodes<NB, P, DIRECT> &codes) {
     constexpr int NCH = P / 8;
@@ -852,10 +838,8 @@ __device__ __forceinline__ void stream_round(const SRow<P> &row, int g, float s,
                         : "r"(bits), "r"(j % CPW == 0 ? 0u : codes.w[j / CPW]), "r"(NB * (j % CPW)), "r"(NB));
                     codes.w[j / CPW] = d;
                 }
-                const bool valid = FULL || (j < g);
-                const float a = fabsf(__fsub_rn(w, what));
-                ar[m] = valid ? a : 0.0f;
-                tm[m] = valid ? __fsub_rn(qf, ws) : 0.0f;  // q - (W - 0)*s
+                ar[m] = fabsf(__fsub_rn(w, what));
+                tm[m] = __fsub_rn(qf, ws);  // q - (W - 0)*s
                 maxr = fmaxf(maxr, ar[m]);
             }
         }
@@ -906,8 +890,8 @@ __device__ __noinline__ float group_zsum_shrink(const __half *wrow, int g, int P
 }
 
 // final codes of a lane's group with the kept zero, written to the packed output
-// [HQQ 算法解读, "第二拍" and "为什么一定要分组"].  DIRECT: the group covers whole 32-bit words
-// of the output, stored as they are.
+// [HQQ 算法解读, "第二拍" and "为什么一定要分组"].  The group covers whole 32-bit words of the
+// output, stored as they are.
 template <int NB, int P>
 __device__ __forceinline__ void group_store_codes(const QParams &Pm, const SRow<P> &row,
                                                   int64_t grp, float s, float z) {
@@ -928,40 +912,11 @@ __device__ __forceinline__ void group_store_codes(const QParams &Pm, const SRow<
     }
 }
 
-// Otherwise the codes are OR-ed into the zeroed output one 32-bit word at a time (a word may
-// be shared with the neighbouring group); clear = true first clears the group's own bits.
-template <int NB>
-__device__ __noinline__ void group_or_codes(const QParams &Pm, const __half *wrow, int64_t grp,
-                                            float s, float z, bool clear) {
-    constexpr int CPW = NB == 4 ? 8 : NB == 2 ? 16 : 10;  // codes per 32-bit word
-    constexpr uint32_t MASK = (1u << NB) - 1u;
-    constexpr float kQmax = (float)((1 << NB) - 1);
-    const int g = Pm.g;
-    const int64_t n0 = grp * g;
-    int64_t wi = n0 / CPW;
-    int c = (int)(n0 - wi * CPW);
-    uint32_t word = 0, mask = 0;
-    uint32_t *out = reinterpret_cast<uint32_t *>(Pm.packed);
-    for (int j = 0; j < g; ++j) {
-        const float t = fminf(fmaxf(__fadd_rn(__fmul_rn(__half2float(wrow[j]), s), z), 0.0f), kQmax);
-        word |= (__float_as_uint(__fadd_rn(t, kMagic)) & MASK) << (NB * c);
-        mask |= MASK << (NB * c);
-        if (++c == CPW || j == g - 1) {  // the packed size is a whole number of words here
-            if (clear) atomicAnd(out + wi, ~mask);
-            atomicOr(out + wi, word);
-            ++wi;
-            c = 0;
-            word = 0;
-            mask = 0;
-        }
-    }
-}
-
-template <int NB, int P, bool FULL>
-__device__ __forceinline__ void group_init(const SRow<P> &row, int g, float eps, float smax,
+template <int NB, int P>
+__device__ __forceinline__ void group_init(const SRow<P> &row, float eps, float smax,
                                            float &s, float &z, float &lo, float &hi) {
     constexpr float kQmax = (float)((1 << NB) - 1);
-    // min and max in fp16 pairs (exact); padded slots repeat element 0
+    // min and max in fp16 pairs (exact)
     __half2 mn2 = *reinterpret_cast<const __half2 *>(&row.h[0]), mx2 = mn2;
 #pragma unroll
     for (int i = 1; i < P / 2; ++i) {
@@ -980,47 +935,26 @@ __device__ __forceinline__ void group_init(const SRow<P> &row, int g, float eps,
     hi = __fmul_rn(mx, s);
 }
 
-// row of group `grp` into registers; slots past g repeat element 0 (inside the group's range)
-template <int P, bool FULL, bool ALIGN16>
-__device__ __forceinline__ void load_row(SRow<P> &row, const __half *W, int64_t grp, int g,
-                                         const __half *slot) {
-    if (ALIGN16) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(slot);
+// row of group `grp` from its shared-memory slot into registers
+template <int P>
+__device__ __forceinline__ void load_row(SRow<P> &row, const __half *slot) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(slot);
 #pragma unroll
-        for (int v = 0; v < P / 8; ++v) {
-            if (FULL || 8 * v < g) {
-                const uint4 x = src[v];
-                row.h[4 * v] = x.x; row.h[4 * v + 1] = x.y; row.h[4 * v + 2] = x.z; row.h[4 * v + 3] = x.w;
-            }
-        }
-    } else {
-        const unsigned short *src = reinterpret_cast<const unsigned short *>(W + grp * g);
-#pragma unroll
-        for (int j = 0; j < P; j += 2) {
-            const uint32_t a = (FULL || j < g) ? src[j] : 0u;
-            const uint32_t b = (FULL || j + 1 < g) ? src[j + 1] : 0u;
-            row.h[j / 2] = a | (b << 16);
-        }
-    }
-    if (!FULL) {
-        const uint32_t e0 = row.h[0] & 0xffffu;
-#pragma unroll
-        for (int j = 0; j < P; ++j)
-            if (j >= g) row.h[j / 2] = (j & 1) ? ((row.h[j / 2] & 0xffffu) | (e0 << 16)) : ((row.h[j / 2] & 0xffff0000u) | e0);
+    for (int v = 0; v < P / 8; ++v) {
+        const uint4 x = src[v];
+        row.h[4 * v] = x.x; row.h[4 * v + 1] = x.y; row.h[4 * v + 2] = x.z; row.h[4 * v + 3] = x.w;
     }
 }
 
-template <int P, bool ALIGN16>
-__device__ __forceinline__ void prefetch_row(__half *slot, const __half *W, int64_t grp, int g) {
-    if (ALIGN16) {
-        const char *src = reinterpret_cast<const char *>(W + grp * g);
-        const uint32_t dst = (uint32_t)__cvta_generic_to_shared(slot);
+// the row of group `grp` (2P bytes, 16-byte aligned) into the lane's slot, asynchronously
+template <int P>
+__device__ __forceinline__ void prefetch_row(__half *slot, const __half *W, int64_t grp) {
+    const char *src = reinterpret_cast<const char *>(W + grp * P);
+    const uint32_t dst = (uint32_t)__cvta_generic_to_shared(slot);
 #pragma unroll
-        for (int v = 0; v < P / 8; ++v)
-            if (8 * v < g)
-                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + 16 * v), "l"(src + 16 * v));
-        asm volatile("cp.async.commit_group;" ::);
-    }
+    for (int v = 0; v < P / 8; ++v)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + 16 * v), "l"(src + 16 * v));
+    asm volatile("cp.async.commit_group;" ::);
 }
 
 __device__ __forceinline__ void prefetch_wait() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
@@ -1046,13 +980,13 @@ __device__ __forceinline__ int64_t claim(const QParams &Pm, bool want) {
     return (want && id < Pm.G) ? id : -1;
 }
 
-template <int NB, int P, bool FULL, bool ALIGN16, bool DIRECT>
+template <int NB, int P>
 __global__ void __launch_bounds__(kThreads) hqq_stream_kernel(const __grid_constant__ QParams Pm) {
     extern __shared__ __align__(16) unsigned char smem[];
     constexpr int NQ = 1 << NB;
     constexpr float kQmax = (float)(NQ - 1);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int K = Pm.K, g = Pm.g;
+    const int K = Pm.K;
     const int Kc = K > 0 ? K : 1;
     float *tabw = reinterpret_cast<float *>(smem) + warp * NQ * 32;
     unsigned *acc = reinterpret_cast<unsigned *>(smem + kWarps * NQ * 32 * 4);
@@ -1068,20 +1002,20 @@ __global__ void __launch_bounds__(kThreads) hqq_stream_kernel(const __grid_const
     for (int i = threadIdx.x; i < K; i += kThreads) { thr_s[i] = Pm.thr[i]; beta_s[i] = Pm.beta[i]; }
     __syncthreads();
     const float thr_last = K > 0 ? thr_s[K - 1] : 0.0f;
-    const float inv_g = 1.0f / (float)g;  // exact for FULL (g = 2^k)
+    constexpr float kInvG = 1.0f / (float)P;  // g = P = 2^k: z = zsum * (1/g) exactly
     const uint32_t tab_adj = (uint32_t)__cvta_generic_to_shared(tabw + lane) - (0x4B400000u << 7);
 
     SRow<P> row;
 #pragma unroll
     for (int i = 0; i < P / 2; ++i) row.h[i] = 0;
-    SCodes<NB, P, DIRECT> codes;
+    SCodes<NB, P, true> codes;
 #pragma unroll
-    for (int i = 0; i < SCodes<NB, P, DIRECT>::kWords; ++i) codes.w[i] = 0;
+    for (int i = 0; i < SCodes<NB, P, true>::kWords; ++i) codes.w[i] = 0;
     float s = 1.0f, z = 0.0f, lo = 0.0f, hi = 0.0f;
     int it = 0;
     int64_t cur = -1;
     int64_t nxt = claim(Pm, true);
-    if (nxt >= 0) prefetch_row<P, ALIGN16>(slot, Pm.W, nxt, g);
+    if (nxt >= 0) prefetch_row<P>(slot, Pm.W, nxt);
     while (true) {
         // ---- a lane without a group takes the prefetched one and prefetches another
         const bool need = cur < 0 && nxt >= 0;
@@ -1089,14 +1023,14 @@ __global__ void __launch_bounds__(kThreads) hqq_stream_kernel(const __grid_const
             if (need) {
                 prefetch_wait();
                 cur = nxt;
-                load_row<P, FULL, ALIGN16>(row, Pm.W, cur, g, slot);
-                group_init<NB, P, FULL>(row, g, Pm.eps_tiny, Pm.scale_max, s, z, lo, hi);
+                load_row<P>(row, slot);
+                group_init<NB, P>(row, Pm.eps_tiny, Pm.scale_max, s, z, lo, hi);
                 it = 0;
             }
             const int64_t n2 = claim(Pm, need);
             if (need) {
                 nxt = n2;
-                if (nxt >= 0) prefetch_row<P, ALIGN16>(slot, Pm.W, nxt, g);
+                if (nxt >= 0) prefetch_row<P>(slot, Pm.W, nxt);
             }
         }
         const bool active = cur >= 0;
@@ -1112,13 +1046,13 @@ __global__ void __launch_bounds__(kThreads) hqq_stream_kernel(const __grid_const
             const bool inside = __fadd_rn(lo, z) >= -0.5f && __fadd_rn(hi, z) < kQmax + 0.5f;
             float esum, zsum, maxr;
             if (__all_sync(kFull, inside))
-                stream_round<NB, P, FULL, false, DIRECT>(row, g, s, z, tab_adj, esum, zsum, maxr, codes);
+                stream_round<NB, P, false, true>(row, s, z, tab_adj, esum, zsum, maxr, codes);
             else
-                stream_round<NB, P, FULL, true, DIRECT>(row, g, s, z, tab_adj, esum, zsum, maxr, codes);
+                stream_round<NB, P, true, true>(row, s, z, tab_adj, esum, zsum, maxr, codes);
             // lp shrink: a residual above the round's safe threshold -> exact binary64 path
             const bool slow = active && maxr > thr_s[ri];
-            if (slow) zsum = group_zsum_shrink<NB>(Pm.W + cur * g, g, P, s, z, tab_adj, beta_s[ri], Pm.p);
-            const float znew = FULL ? __fmul_rn(zsum, inv_g) : __fdiv_rn(zsum, (float)g);
+            if (slow) zsum = group_zsum_shrink<NB>(Pm.W + cur * P, P, P, s, z, tab_adj, beta_s[ri], Pm.p);
+            const float znew = __fmul_rn(zsum, kInvG);
             if (active && K > 0) {
                 const bool frozen = !slow && !(maxr > thr_last) && (znew == z);
                 done = frozen || it == K - 1;
@@ -1134,16 +1068,12 @@ __global__ void __launch_bounds__(kThreads) hqq_stream_kernel(const __grid_const
         if (done) {
             // the codes of a group's last round are its final codes (z is the kept zero);
             // with no round at all they are computed here
-            if constexpr (DIRECT) {
-                if (K == 0) {
-                    group_store_codes<NB, P>(Pm, row, cur, s, z);
-                } else {
-                    uint32_t *dst = reinterpret_cast<uint32_t *>(Pm.packed) + cur * (P * NB / 32);
-#pragma unroll
-                    for (int i = 0; i < SCodes<NB, P, DIRECT>::kWords; ++i) dst[i] = codes.w[i];
-                }
+            if (K == 0) {
+                group_store_codes<NB, P>(Pm, row, cur, s, z);
             } else {
-                group_or_codes<NB>(Pm, Pm.W + cur * g, cur, s, z, false);
+                uint32_t *dst = reinterpret_cast<uint32_t *>(Pm.packed) + cur * (P * NB / 32);
+#pragma unroll
+                for (int i = 0; i < SCodes<NB, P, true>::kWords; ++i) dst[i] = codes.w[i];
             }
             write_meta(Pm, cur, s, z, it);
             cur = -1;
@@ -1179,11 +1109,11 @@ __global__ void __launch_bounds__(kThreads) hqq_stream_kernel(const __grid_const
 
 // Groups whose own last round f lies past the kept round b make exactly min(b, f) zero
 // updates again and rewrite their codes and metadata.  Nothing to do when b = iters - 1.
-template <int NB, int P, bool FULL, bool ALIGN16, bool DIRECT>
+template <int NB, int P>
 __global__ void __launch_bounds__(kThreads) hqq_stream_fixup_kernel(const __grid_constant__ QParams Pm) {
     extern __shared__ __align__(16) unsigned char smem[];
     constexpr int NQ = 1 << NB;
-    const int K = Pm.K, g = Pm.g;
+    const int K = Pm.K;
     const int b = __ldcg(&ctl_of(Pm)->b);
     if (K == 0 || b >= K - 1) return;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -1200,25 +1130,8 @@ __global__ void __launch_bounds__(kThreads) hqq_stream_fixup_kernel(const __grid
         for (int i = 0; i < P / 2; ++i) row.h[i] = 0;
         float s = 1.0f, z = 0.0f, lo = 0.0f, hi = 0.0f;
         if (stale) {
-            if (ALIGN16) {  // synchronous load of the row
-                const uint4 *src = reinterpret_cast<const uint4 *>(Pm.W + grp * g);
-#pragma unroll
-                for (int v = 0; v < P / 8; ++v) {
-                    if (FULL || 8 * v < g) {
-                        const uint4 x = src[v];
-                        row.h[4 * v] = x.x; row.h[4 * v + 1] = x.y; row.h[4 * v + 2] = x.z; row.h[4 * v + 3] = x.w;
-                    }
-                }
-                if (!FULL) {
-                    const uint32_t e0 = row.h[0] & 0xffffu;
-#pragma unroll
-                    for (int j = 0; j < P; ++j)
-                        if (j >= g) row.h[j / 2] = (j & 1) ? ((row.h[j / 2] & 0xffffu) | (e0 << 16)) : ((row.h[j / 2] & 0xffff0000u) | e0);
-                }
-            } else {
-                load_row<P, FULL, false>(row, Pm.W, grp, g, nullptr);
-            }
-            group_init<NB, P, FULL>(row, g, Pm.eps_tiny, Pm.scale_max, s, z, lo, hi);
+            load_row<P>(row, Pm.W + grp * P);  // synchronous: the row is read once
+            group_init<NB, P>(row, Pm.eps_tiny, Pm.scale_max, s, z, lo, hi);
         }
         const int n = stale ? min(b, f) : 0;
         for (int r = 0; __any_sync(kFull, r < n); ++r) {
@@ -1226,16 +1139,15 @@ __global__ void __launch_bounds__(kThreads) hqq_stream_fixup_kernel(const __grid
             for (int k = 0; k < NQ; ++k) tabw[k * 32 + lane] = __fdiv_rn(__fsub_rn((float)k, z), s);
             float esum, zsum, maxr;
             SCodes<NB, P, false> nocodes;
-            stream_round<NB, P, FULL, true, false>(row, g, s, z, tab_adj, esum, zsum, maxr, nocodes);
+            stream_round<NB, P, true, false>(row, s, z, tab_adj, esum, zsum, maxr, nocodes);
             const int rr = min(r, K - 1);
             const bool slow = r < n && maxr > Pm.thr[rr];
-            if (slow) zsum = group_zsum_shrink<NB>(Pm.W + grp * g, g, P, s, z, tab_adj, Pm.beta[rr], Pm.p);
-            const float znew = FULL ? __fmul_rn(zsum, 1.0f / (float)g) : __fdiv_rn(zsum, (float)g);
+            if (slow) zsum = group_zsum_shrink<NB>(Pm.W + grp * P, P, P, s, z, tab_adj, Pm.beta[rr], Pm.p);
+            const float znew = __fmul_rn(zsum, 1.0f / (float)P);
             if (r < n) z = znew;
         }
         if (stale) {
-            if constexpr (DIRECT) group_store_codes<NB, P>(Pm, row, grp, s, z);
-            else group_or_codes<NB>(Pm, Pm.W + grp * g, grp, s, z, true);
+            group_store_codes<NB, P>(Pm, row, grp, s, z);
             write_meta(Pm, grp, s, z, -1);
         }
     }
@@ -1511,11 +1423,11 @@ cudaError_t launch_quant_l(const QParams &P, int L, int64_t ntiles, cudaStream_t
     }
 }
 
-template <int NB, int P, bool FULL, bool ALIGN16, bool DIRECT>
+template <int NB, int P>
 cudaError_t launch_stream(const QParams &Pm, cudaStream_t st) {
     const int smem = StreamSmem::bytes(P, 1 << NB, Pm.K);
-    auto k1 = hqq_stream_kernel<NB, P, FULL, ALIGN16, DIRECT>;
-    auto k2 = hqq_stream_fixup_kernel<NB, P, FULL, ALIGN16, DIRECT>;
+    auto k1 = hqq_stream_kernel<NB, P>;
+    auto k2 = hqq_stream_fixup_kernel<NB, P>;
     cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -1529,8 +1441,6 @@ cudaError_t launch_stream(const QParams &Pm, cudaStream_t st) {
     const int64_t lanes_needed = (Pm.G + 31) / 32 * 32;
     const unsigned blocks = (unsigned)std::max<int64_t>(
         1, std::min<int64_t>((int64_t)sms * per_sm, (lanes_needed + kThreads - 1) / kThreads));
-    if (!DIRECT && cudaMemsetAsync(Pm.packed, 0, Pm.packed_bytes, st) != cudaSuccess)
-        return cudaGetLastError();
     k1<<<blocks, kThreads, smem, st>>>(Pm);
     const unsigned fix_blocks = (unsigned)std::min<int64_t>((int64_t)sms * per_sm,
                                                             (Pm.G + kThreads - 1) / kThreads);
@@ -1541,10 +1451,10 @@ cudaError_t launch_stream(const QParams &Pm, cudaStream_t st) {
 template <int NB>
 cudaError_t launch_stream_nb(const QParams &Pm, int P, cudaStream_t st) {
     switch (P) {
-    case 16: return launch_stream<NB, 16, true, true, true>(Pm, st);
-    case 32: return launch_stream<NB, 32, true, true, true>(Pm, st);
-    case 64: return launch_stream<NB, 64, true, true, true>(Pm, st);
-    default: return launch_stream<NB, 128, true, true, true>(Pm, st);
+    case 16: return launch_stream<NB, 16>(Pm, st);
+    case 32: return launch_stream<NB, 32>(Pm, st);
+    case 64: return launch_stream<NB, 64>(Pm, st);
+    default: return launch_stream<NB, 128>(Pm, st);
     }
 }
 

@@ -202,6 +202,7 @@ __device__ void init_tile(const QParams &P, const __half *wh, float *s_t, float 
     for (int i = threadIdx.x; i < tg; i += kThreads) {
         const __half *row = wh + i * P.stride;
         float mn[4], mx[4];
+        bool nan = false;
 #pragma unroll
         for (int c = 0; c < 4; ++c) { mn[c] = INFINITY; mx[c] = -INFINITY; }
         int j = 0;
@@ -211,12 +212,14 @@ __device__ void init_tile(const QParams &P, const __half *wh, float *s_t, float 
                 const float v = __half2float(row[j + c]);
                 mn[c] = fminf(mn[c], v);
                 mx[c] = fmaxf(mx[c], v);
+                nan |= v != v;
             }
         }
         for (; j < g; ++j) {
             const float v = __half2float(row[j]);
             mn[0] = fminf(mn[0], v);
             mx[0] = fmaxf(mx[0], v);
+            nan |= v != v;
         }
         const float lo_w = fminf(fminf(mn[0], mn[1]), fminf(mn[2], mn[3]));
         const float hi_w = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
@@ -225,7 +228,9 @@ __device__ void init_tile(const QParams &P, const __half *wh, float *s_t, float 
         s = fminf(s, P.scale_max);
         s_t[i] = s;
         z_t[i] = __fsub_rn(0.0f, __fmul_rn(lo_w, s));
-        lo_t[i] = __fmul_rn(lo_w, s);
+        // a NaN in the group sends its warp down the clamped path (fmaxf(NaN, 0) = 0), so
+        // table addresses stay in range whatever W holds
+        lo_t[i] = nan ? __int_as_float(0x7fc00000) : __fmul_rn(lo_w, s);
         hi_t[i] = __fmul_rn(hi_w, s);
     }
 }
@@ -758,22 +763,45 @@ __global__ void __launch_bounds__(kThreads, 2) hqq_fixup_kernel(const __grid_con
 }
 
 // ==========================================================================================
-// Streaming engine (axis 1): one lane per group
+// Streaming engine (axis 1; 2- or 4-bit codes; power-of-two groups of 16 .. 128 elements that
+// fill whole 32-bit words of the output): one lane per group
 //
 // Each lane holds one whole group: its fp16 row in registers (P/2 words), its own table of the
 // 2^b reconstructions in a private shared-memory column, and its running state.  Lanes take
 // groups from a global counter (one atomic per warp and refill), so the work stays balanced
 // to the end, and each lane copies its next group's row into a shared-memory slot with
-// cp.async one group ahead.  The pairwise group sums are an 8-element tree per chunk and a
-// compile-time stack over the chunks; no shuffles are needed.
+// cp.async one group ahead.
+//
+// The arithmetic runs on packed binary32 pairs (add/mul/fma.rn.f32x2: two IEEE operations per
+// instruction, each rounded exactly as its scalar form).  A register word pairs element j with
+// element j + 8 of the same 16-element block, so the two halves of every pair fall in two
+// consecutive 8-element chunks.  The pairwise tree of each chunk then runs on both chunks at
+// once, and the group sums keep the oracle's order: an 8-element tree per chunk, then
+// recursive halving over the chunks.
 // ==========================================================================================
 template <int P>
 struct SRow {
-    uint32_t h[P / 2];  // fp16 pairs: element 2i in the low half
+    uint32_t h[P / 2];  // word 8c + m: element 16c + m (low half) and 16c + 8 + m (high half)
 };
 
 __device__ __forceinline__ float half_lo(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v & 0xffffu))); }
 __device__ __forceinline__ float half_hi(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v >> 16))); }
+
+// element j of a row held in the paired layout
+template <int P>
+__device__ __forceinline__ float row_elem(const SRow<P> &row, int j) {
+    const uint32_t w = row.h[(j >> 4) * 8 + (j & 7)];
+    return (j & 8) ? half_hi(w) : half_lo(w);
+}
+
+// one 16-element block from its natural fp16 words n[i] = (x[2i], x[2i+1]) to the paired layout
+__device__ __forceinline__ void pair_block(uint32_t *dst, uint32_t n0, uint32_t n1, uint32_t n2,
+                                           uint32_t n3, uint32_t n4, uint32_t n5, uint32_t n6,
+                                           uint32_t n7) {
+    const uint32_t lo[4] = {n0, n1, n2, n3}, hi[4] = {n4, n5, n6, n7};
+#pragma unroll
+    for (int m = 0; m < 8; ++m) dst[m] = __byte_perm(lo[m >> 1], hi[m >> 1], (m & 1) ? 0x7632 : 0x5410);
+}
 
 // push a chunk's sum onto a pairwise stack: after chunk ch, level l holds the sum of the last
 // 2^l chunks whenever bit l of ch + 1 is set; the final entry is the whole pairwise sum
@@ -795,56 +823,126 @@ __device__ __forceinline__ float tree8(const float *x) {
                      __fadd_rn(__fadd_rn(x[4], x[5]), __fadd_rn(x[6], x[7])));
 }
 
+// the 8-element pairwise trees of two chunks at once (x[m] = element m of each chunk)
+__device__ __forceinline__ float2 tree8x2(const float2 *x) {
+    return __fadd2_rn(__fadd2_rn(__fadd2_rn(x[0], x[1]), __fadd2_rn(x[2], x[3])),
+                      __fadd2_rn(__fadd2_rn(x[4], x[5]), __fadd2_rn(x[6], x[7])));
+}
+
+// the same for |x|: the first level in scalar adds, which take |.| for free
+__device__ __forceinline__ float2 abs_tree8x2(const float2 *x) {
+    float2 l1[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        l1[i] = make_float2(__fadd_rn(fabsf(x[2 * i].x), fabsf(x[2 * i + 1].x)),
+                            __fadd_rn(fabsf(x[2 * i].y), fabsf(x[2 * i + 1].y)));
+    return __fadd2_rn(__fadd2_rn(l1[0], l1[1]), __fadd2_rn(l1[2], l1[3]));
+}
+
+__device__ __forceinline__ void sts_f32(uint32_t addr, float v) {
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v));
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    return v;
+}
+
+// The reconstructions W_hat_k = (k - z)/s of every code k [HQQ 算法解读, "第二拍"], correctly
+// rounded, into this lane's table column (entry k at col + 128 k).  Each quotient is
+// (k - z) * y with y = RN(1/s), refined by two remainder corrections q + RN(a - s q) * y
+// (Markstein, IBM J. Res. Dev. 34(1), 1990: with y = RN(1/s) and q within one ulp of a/s,
+// the correction rounds to RN(a/s)).  The first correction brings the product within one
+// ulp; the second then rounds it.  The quotients must lie in the normal range: with
+// |z| >= 2^-60 (or z = 0), every nonzero |k - z|/s exceeds 2^-80 for s <= 2^15.  Otherwise
+// the lane divides.
+template <int NQ>
+__device__ __forceinline__ void build_table(uint32_t col, float s, float y, float z) {
+    if (z == 0.0f || fabsf(z) >= 0x1p-60f) {
+        const float2 y2 = make_float2(y, y), ns2 = make_float2(-s, -s), nz2 = make_float2(-z, -z);
+#pragma unroll
+        for (int k = 0; k < NQ; k += 2) {
+            const float2 a = __fadd2_rn(make_float2((float)k, (float)(k + 1)), nz2);  // k - z
+            const float2 q0 = __fmul2_rn(a, y2);
+            const float2 q1 = __ffma2_rn(__ffma2_rn(q0, ns2, a), y2, q0);
+            const float2 q2 = __ffma2_rn(__ffma2_rn(q1, ns2, a), y2, q1);
+            sts_f32(col + 128u * k, q2.x);
+            sts_f32(col + 128u * (k + 1), q2.y);
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < NQ; ++k) sts_f32(col + 128u * k, __fdiv_rn(__fsub_rn((float)k, z), s));
+    }
+}
+
+// An upper bound on every |RN(W - W_hat)| of the round, from the group's state alone:
+// lz = RN(lo + z) and hz = RN(hi + z) are the smallest and largest W s + z of the group, so
+// |t - q| <= max(1/2, -lz, hz - qmax).  The rounding of W s, of + z, of the table and of the
+// difference adds less than (3A + 4|z| + 3 qmax) 2^-24 with A = max(|lo|, |hi|), and the
+// bound is taken twice that wide and scaled by 1 + 2^-20 to cover its own rounding.
+__device__ __forceinline__ float resid_bound(float lz, float hz, float A, float z, float y,
+                                             float qmax) {
+    const float M = fmaxf(0.5f, fmaxf(-lz, __fsub_rn(hz, qmax)));
+    const float slack = __fmul_rn(__fadd_rn(__fmul_rn(8.0f, __fadd_rn(A, fabsf(z))), 4.0f * qmax), 0x1p-23f);
+    return __fmul_rn(__fmul_rn(__fadd_rn(M, slack), y), 1.0f + 0x1p-20f);
+}
+
 template <int NB, int P, bool DIRECT>
 struct SCodes {  // a lane's codes of the current round, in the output's packed format
     static constexpr int kWords = DIRECT ? P * NB / 32 : 1;
     uint32_t w[kWords];
+    __device__ __forceinline__ void put(int j, uint32_t bits) {  // code j: low NB bits of bits
+        constexpr int CPW = 32 / NB;
+        uint32_t d;
+        asm("bfi.b32 %0, %1, %2, %3, %4;" : "=r"(d)
+            : "r"(bits), "r"(j % CPW == 0 ? 0u : w[j / CPW]), "r"(NB * (j % CPW)), "r"(NB));
+        w[j / CPW] = d;
+    }
 };
 
 // One proximal round over a lane's group [HQQ 算法解读, "第二拍"] with e = 0 for every element.
-// Returns the group's error sum, the zero-update sum (z_new times g), the largest residual
-// and (DIRECT) the round's codes.  CLIP: clamp W*s + z to [0, 2^b - 1] before rounding.
+// Returns the group's error sum, the zero-update sum (z_new times g) and (DIRECT) the round's
+// codes.  CLIP: clamp W s + z to [0, 2^b - 1] before rounding.
 template <int NB, int P, bool CLIP, bool DIRECT>
 __device__ __forceinline__ void stream_round(const SRow<P> &row, float s, float z,
                                              uint32_t tab_adj, float &esum, float &zsum,
-                                             float &maxr, SCodes<NB, P, DIRECT> &codes) {
+                                             SCodes<NB, P, DIRECT> &codes) {
     constexpr int NCH = P / 8;
-    constexpr int LOGN = NCH == 1 ? 0 : NCH == 2 ? 1 : NCH == 4 ? 2 : NCH == 8 ? 3 : NCH == 16 ? 4 : 5;
+    constexpr int LOGN = NCH == 2 ? 1 : NCH == 4 ? 2 : NCH == 8 ? 3 : 4;
     constexpr float kQmax = (float)((1 << NB) - 1);
+    const float2 s2 = make_float2(s, s), z2 = make_float2(z, z);
+    const float2 mg2 = make_float2(kMagic, kMagic), nmg2 = make_float2(-kMagic, -kMagic);
+    const float2 neg1 = make_float2(-1.0f, -1.0f);
     float sa[LOGN + 1], st[LOGN + 1];
-    maxr = 0.0f;
 #pragma unroll
-    for (int ch = 0; ch < NCH; ++ch) {
-        float ar[8], tm[8];
+    for (int c = 0; c < P / 16; ++c) {
+        float2 d[8], tm[8];
 #pragma unroll
-        for (int m2 = 0; m2 < 8; m2 += 2) {
-            const float2 wp = __half22float2(*reinterpret_cast<const __half2 *>(&row.h[(8 * ch + m2) / 2]));
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int m = m2 + h, j = 8 * ch + m;
-                const float w = h ? wp.y : wp.x;
-                const float ws = __fmul_rn(w, s);
-                float t = __fadd_rn(ws, z);
-                if (CLIP) t = fminf(fmaxf(t, 0.0f), kQmax);
-                const float u = __fadd_rn(t, kMagic);
-                const float qf = __fsub_rn(u, kMagic);
-                const uint32_t bits = __float_as_uint(u);
-                float what;
-                asm volatile("ld.shared.f32 %0, [%1];" : "=f"(what) : "r"(tab_adj + (bits << 7)));
-                if (DIRECT) {  // code j at bit NB*j of the group's words (low NB bits of `bits`)
-                    constexpr int CPW = 32 / NB;
-                    uint32_t d;
-                    asm("bfi.b32 %0, %1, %2, %3, %4;" : "=r"(d)
-                        : "r"(bits), "r"(j % CPW == 0 ? 0u : codes.w[j / CPW]), "r"(NB * (j % CPW)), "r"(NB));
-                    codes.w[j / CPW] = d;
-                }
-                ar[m] = fabsf(__fsub_rn(w, what));
-                tm[m] = __fsub_rn(qf, ws);  // q - (W - 0)*s
-                maxr = fmaxf(maxr, ar[m]);
+        for (int m = 0; m < 8; ++m) {
+            const float2 w = __half22float2(*reinterpret_cast<const __half2 *>(&row.h[8 * c + m]));
+            const float2 ws = __fmul2_rn(w, s2);
+            float2 t = __fadd2_rn(ws, z2);
+            if (CLIP) {
+                t.x = fminf(fmaxf(t.x, 0.0f), kQmax);
+                t.y = fminf(fmaxf(t.y, 0.0f), kQmax);
             }
+            const float2 u = __fadd2_rn(t, mg2);     // round half to even: the integer in the
+            const float2 qf = __fadd2_rn(u, nmg2);   // low mantissa bits of u
+            const uint32_t ba = __float_as_uint(u.x), bb = __float_as_uint(u.y);
+            const float2 what = make_float2(lds_f32(tab_adj + (ba << 7)), lds_f32(tab_adj + (bb << 7)));
+            if (DIRECT) {
+                codes.put(16 * c + m, ba);
+                codes.put(16 * c + 8 + m, bb);
+            }
+            d[m] = __ffma2_rn(what, neg1, w);   // W - W_hat
+            tm[m] = __ffma2_rn(ws, neg1, qf);   // q - (W - 0) s
         }
-        pw_push<LOGN>(sa, ch, tree8(ar));
-        pw_push<LOGN>(st, ch, tree8(tm));
+        const float2 ea = abs_tree8x2(d), ta = tree8x2(tm);
+        pw_push<LOGN>(sa, 2 * c, ea.x);
+        pw_push<LOGN>(sa, 2 * c + 1, ea.y);
+        pw_push<LOGN>(st, 2 * c, ta.x);
+        pw_push<LOGN>(st, 2 * c + 1, ta.y);
     }
     esum = sa[LOGN];
     zsum = st[LOGN];
@@ -872,8 +970,7 @@ __device__ __noinline__ float group_zsum_shrink(const __half *wrow, int g, int P
                 const float t = fminf(fmaxf(__fadd_rn(__fmul_rn(w, s), z), 0.0f), kQmax);
                 const float u = __fadd_rn(t, kMagic);
                 const float qf = __fsub_rn(u, kMagic);
-                float what;
-                asm volatile("ld.shared.f32 %0, [%1];" : "=f"(what) : "r"(tab_adj + (__float_as_uint(u) << 7)));
+                const float what = lds_f32(tab_adj + (__float_as_uint(u) << 7));
                 const float e = shrink_lp(__fsub_rn(w, what), beta, p);
                 term = __fsub_rn(qf, __fmul_rn(__fsub_rn(w, e), s));
             }
@@ -903,8 +1000,7 @@ __device__ __forceinline__ void group_store_codes(const QParams &Pm, const SRow<
         uint32_t word = 0;
 #pragma unroll
         for (int c = 0; c < CPW; ++c) {
-            const int j = wi * CPW + c;
-            const float w = (j & 1) ? half_hi(row.h[j / 2]) : half_lo(row.h[j / 2]);
+            const float w = row_elem<P>(row, wi * CPW + c);
             const float t = fminf(fmaxf(__fadd_rn(__fmul_rn(w, s), z), 0.0f), kQmax);
             word |= (__float_as_uint(__fadd_rn(t, kMagic)) & ((1u << NB) - 1u)) << (NB * c);
         }
@@ -912,52 +1008,86 @@ __device__ __forceinline__ void group_store_codes(const QParams &Pm, const SRow<
     }
 }
 
+// the group's metadata [HQQ 算法解读, "量化公式"]: Delta = 1/s (y = RN(1/s)) and z in fp16
+__device__ __forceinline__ void stream_meta(const QParams &Pm, int64_t k, float s, float y,
+                                            float z, int f) {
+    Pm.scale[k] = __float2half_rn(y);
+    Pm.zero[k] = __float2half_rn(z);
+    if (Pm.s_out) Pm.s_out[k] = s;
+    if (Pm.z_out) Pm.z_out[k] = z;
+    if (f >= 0) {
+        Pm.fk[k] = (uint8_t)f;
+        if (Pm.group_rounds) Pm.group_rounds[k] = Pm.K > 0 ? (uint8_t)(f + 1) : 0;
+    }
+}
+
+// per-group state of the streaming engine
+struct SGroup {
+    float s, y, z, lo, hi, A;  // scale, RN(1/s), zero, min*s, max*s, max(|lo|, |hi|)
+    __device__ __forceinline__ void idle() { s = 1.0f; y = 1.0f; z = 0.0f; lo = 0.0f; hi = 0.0f; A = 0.0f; }
+};
+
 template <int NB, int P>
-__device__ __forceinline__ void group_init(const SRow<P> &row, float eps, float smax,
-                                           float &s, float &z, float &lo, float &hi) {
+__device__ __forceinline__ void group_init(const SRow<P> &row, float eps, float smax, SGroup &gs) {
     constexpr float kQmax = (float)((1 << NB) - 1);
-    // min and max in fp16 pairs (exact)
+    // min and max in fp16 pairs (exact).  A NaN propagates into lo and hi, which sends the
+    // warp down the clamped path (fmaxf(NaN, 0) = 0): table addresses stay in range whatever
+    // W holds
     __half2 mn2 = *reinterpret_cast<const __half2 *>(&row.h[0]), mx2 = mn2;
 #pragma unroll
     for (int i = 1; i < P / 2; ++i) {
         const __half2 v = *reinterpret_cast<const __half2 *>(&row.h[i]);
-        mn2 = __hmin2(mn2, v);
-        mx2 = __hmax2(mx2, v);
+        mn2 = __hmin2_nan(mn2, v);
+        mx2 = __hmax2_nan(mx2, v);
     }
     const float mn = fminf(__low2float(mn2), __high2float(mn2));
     const float mx = fmaxf(__low2float(mx2), __high2float(mx2));
     // [HQQ 算法解读, "第一拍：min-max 给一个可用的初值"]
     const float d = __fsub_rn(mx, mn);
-    s = (d < eps) ? 1.0f : __fdiv_rn(kQmax, d);
+    float s = (d < eps) ? 1.0f : __fdiv_rn(kQmax, d);
     s = fminf(s, smax);
-    z = __fsub_rn(0.0f, __fmul_rn(mn, s));
-    lo = __fmul_rn(mn, s);
-    hi = __fmul_rn(mx, s);
+    gs.s = s;
+    gs.y = __frcp_rn(s);
+    gs.z = __fsub_rn(0.0f, __fmul_rn(mn, s));
+    gs.lo = __fmul_rn(mn, s);
+    gs.hi = __fmul_rn(mx, s);
+    gs.A = fmaxf(fabsf(gs.lo), fabsf(gs.hi));
 }
 
-// row of group `grp` from its shared-memory slot into registers
+// the row of a group into registers, in the paired layout.  From the lane's shared-memory
+// slot, where 16-byte chunk v sits at position v ^ sw (the swizzle spreads the lanes of a
+// quarter warp over all banks), or (sw < 0) straight from global memory.
 template <int P>
-__device__ __forceinline__ void load_row(SRow<P> &row, const __half *slot) {
-    const uint4 *src = reinterpret_cast<const uint4 *>(slot);
+__device__ __forceinline__ void load_row(SRow<P> &row, const __half *src_row, int sw) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(src_row);
 #pragma unroll
-    for (int v = 0; v < P / 8; ++v) {
-        const uint4 x = src[v];
-        row.h[4 * v] = x.x; row.h[4 * v + 1] = x.y; row.h[4 * v + 2] = x.z; row.h[4 * v + 3] = x.w;
+    for (int c = 0; c < P / 16; ++c) {
+        const uint4 a = src[sw < 0 ? 2 * c : (2 * c) ^ sw];
+        const uint4 b = src[sw < 0 ? 2 * c + 1 : (2 * c + 1) ^ sw];
+        pair_block(&row.h[8 * c], a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w);
     }
 }
 
 // the row of group `grp` (2P bytes, 16-byte aligned) into the lane's slot, asynchronously
 template <int P>
-__device__ __forceinline__ void prefetch_row(__half *slot, const __half *W, int64_t grp) {
+__device__ __forceinline__ void prefetch_row(__half *slot, const __half *W, int64_t grp, int sw) {
     const char *src = reinterpret_cast<const char *>(W + grp * P);
     const uint32_t dst = (uint32_t)__cvta_generic_to_shared(slot);
 #pragma unroll
     for (int v = 0; v < P / 8; ++v)
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + 16 * v), "l"(src + 16 * v));
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + 16 * (v ^ sw)), "l"(src + 16 * v));
     asm volatile("cp.async.commit_group;" ::);
 }
 
 __device__ __forceinline__ void prefetch_wait() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// the slot swizzle of a lane: the P/8 chunks of lanes l .. l+7 (one quarter warp of 16-byte
+// accesses) must land in 8 different 16-byte bank groups
+template <int P>
+__device__ __forceinline__ int slot_swizzle(int lane) {
+    constexpr int C = P / 8;  // chunks per slot: 2, 4, 8 or 16
+    return C >= 8 ? (lane & 7) : C == 4 ? ((lane >> 1) & 3) : ((lane >> 2) & 1);
+}
 
 struct StreamSmem {
     static __host__ __device__ int bytes(int P, int nq, int K) {
@@ -1003,7 +1133,9 @@ __global__ void __launch_bounds__(kThreads) hqq_stream_kernel(const __grid_const
     __syncthreads();
     const float thr_last = K > 0 ? thr_s[K - 1] : 0.0f;
     constexpr float kInvG = 1.0f / (float)P;  // g = P = 2^k: z = zsum * (1/g) exactly
-    const uint32_t tab_adj = (uint32_t)__cvta_generic_to_shared(tabw + lane) - (0x4B400000u << 7);
+    const uint32_t col = (uint32_t)__cvta_generic_to_shared(tabw + lane);
+    const uint32_t tab_adj = col - (0x4B400000u << 7);
+    const int sw = slot_swizzle<P>(lane);
 
     SRow<P> row;
 #pragma unroll
@@ -1011,11 +1143,12 @@ __global__ void __launch_bounds__(kThreads) hqq_stream_kernel(const __grid_const
     SCodes<NB, P, true> codes;
 #pragma unroll
     for (int i = 0; i < SCodes<NB, P, true>::kWords; ++i) codes.w[i] = 0;
-    float s = 1.0f, z = 0.0f, lo = 0.0f, hi = 0.0f;
+    SGroup gs;
+    gs.idle();
     int it = 0;
     int64_t cur = -1;
     int64_t nxt = claim(Pm, true);
-    if (nxt >= 0) prefetch_row<P>(slot, Pm.W, nxt);
+    if (nxt >= 0) prefetch_row<P>(slot, Pm.W, nxt, sw);
     while (true) {
         // ---- a lane without a group takes the prefetched one and prefetches another
         const bool need = cur < 0 && nxt >= 0;
@@ -1023,14 +1156,14 @@ __global__ void __launch_bounds__(kThreads) hqq_stream_kernel(const __grid_const
             if (need) {
                 prefetch_wait();
                 cur = nxt;
-                load_row<P>(row, slot);
-                group_init<NB, P>(row, Pm.eps_tiny, Pm.scale_max, s, z, lo, hi);
+                load_row<P>(row, slot, sw);
+                group_init<NB, P>(row, Pm.eps_tiny, Pm.scale_max, gs);
                 it = 0;
             }
             const int64_t n2 = claim(Pm, need);
             if (need) {
                 nxt = n2;
-                if (nxt >= 0) prefetch_row<P>(slot, Pm.W, nxt);
+                if (nxt >= 0) prefetch_row<P>(slot, Pm.W, nxt, sw);
             }
         }
         const bool active = cur >= 0;
@@ -1038,29 +1171,28 @@ __global__ void __launch_bounds__(kThreads) hqq_stream_kernel(const __grid_const
         bool done = active && K == 0;
         if (__any_sync(kFull, active && K > 0)) {
             const int ri = min(it, max(K - 1, 0));
-            // the reconstructions W_hat = (k - z)/s of every code k, in this lane's column
-#pragma unroll
-            for (int k = 0; k < NQ; ++k) tabw[k * 32 + lane] = __fdiv_rn(__fsub_rn((float)k, z), s);
-            // no clip is needed when [lo + z, hi + z] rounds inside [0, 2^b - 1]; lanes without
-            // a group hold a zero row and zero state
-            const bool inside = __fadd_rn(lo, z) >= -0.5f && __fadd_rn(hi, z) < kQmax + 0.5f;
-            float esum, zsum, maxr;
+            build_table<NQ>(col, gs.s, gs.y, gs.z);
+            // no clip is needed when [lo + z, hi + z] rounds inside [0, 2^b - 1]; a lane without
+            // a group holds a zero row and zero state, or its last group's row and state
+            const float lz = __fadd_rn(gs.lo, gs.z), hz = __fadd_rn(gs.hi, gs.z);
+            const bool inside = lz >= -0.5f && hz < kQmax + 0.5f;
+            float esum, zsum;
             if (__all_sync(kFull, inside))
-                stream_round<NB, P, false, true>(row, s, z, tab_adj, esum, zsum, maxr, codes);
+                stream_round<NB, P, false, true>(row, gs.s, gs.z, tab_adj, esum, zsum, codes);
             else
-                stream_round<NB, P, true, true>(row, s, z, tab_adj, esum, zsum, maxr, codes);
-            // lp shrink: a residual above the round's safe threshold -> exact binary64 path
-            const bool slow = active && maxr > thr_s[ri];
-            if (slow) zsum = group_zsum_shrink<NB>(Pm.W + cur * P, P, P, s, z, tab_adj, beta_s[ri], Pm.p);
+                stream_round<NB, P, true, true>(row, gs.s, gs.z, tab_adj, esum, zsum, codes);
+            // lp shrink: a residual that may exceed the round's safe threshold -> exact binary64
+            const float B = resid_bound(lz, hz, gs.A, gs.z, gs.y, kQmax);
+            const bool slow = active && B > thr_s[ri];
+            if (slow) zsum = group_zsum_shrink<NB>(Pm.W + cur * P, P, P, gs.s, gs.z, tab_adj, beta_s[ri], Pm.p);
             const float znew = __fmul_rn(zsum, kInvG);
             if (active && K > 0) {
-                const bool frozen = !slow && !(maxr > thr_last) && (znew == z);
-                done = frozen || it == K - 1;
+                done = (!slow && !(B > thr_last) && znew == gs.z) || it == K - 1;
                 const u64 fx = err_fixed(esum);
                 add_fixed(acc_w + 4 * it, fx);
                 if (done && it + 1 < K) add_fixed(acc_w + 4 * (K + it + 1), fx);
                 if (!done) {
-                    z = znew;
+                    gs.z = znew;
                     ++it;
                 }
             }
@@ -1069,18 +1201,16 @@ __global__ void __launch_bounds__(kThreads) hqq_stream_kernel(const __grid_const
             // the codes of a group's last round are its final codes (z is the kept zero);
             // with no round at all they are computed here
             if (K == 0) {
-                group_store_codes<NB, P>(Pm, row, cur, s, z);
+                group_store_codes<NB, P>(Pm, row, cur, gs.s, gs.z);
             } else {
                 uint32_t *dst = reinterpret_cast<uint32_t *>(Pm.packed) + cur * (P * NB / 32);
 #pragma unroll
                 for (int i = 0; i < SCodes<NB, P, true>::kWords; ++i) dst[i] = codes.w[i];
             }
-            write_meta(Pm, cur, s, z, it);
+            stream_meta(Pm, cur, gs.s, gs.y, gs.z, it);
+            // the lane keeps its finished group's row and state until it takes the next one:
+            // the pair stays consistent, so its rounds stay inside the table
             cur = -1;
-            // an idle lane holds a zero row and zero state, inside every range
-#pragma unroll
-            for (int i = 0; i < P / 2; ++i) row.h[i] = 0;
-            s = 1.0f; z = 0.0f; lo = 0.0f; hi = 0.0f;
         }
     }
     // this warp's per-round sums (16-bit chunks) -> 128-bit global sums
@@ -1113,12 +1243,14 @@ template <int NB, int P>
 __global__ void __launch_bounds__(kThreads) hqq_stream_fixup_kernel(const __grid_constant__ QParams Pm) {
     extern __shared__ __align__(16) unsigned char smem[];
     constexpr int NQ = 1 << NB;
+    constexpr float kQmax = (float)(NQ - 1);
     const int K = Pm.K;
     const int b = __ldcg(&ctl_of(Pm)->b);
     if (K == 0 || b >= K - 1) return;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     float *tabw = reinterpret_cast<float *>(smem) + warp * NQ * 32;
-    const uint32_t tab_adj = (uint32_t)__cvta_generic_to_shared(tabw + lane) - (0x4B400000u << 7);
+    const uint32_t col = (uint32_t)__cvta_generic_to_shared(tabw + lane);
+    const uint32_t tab_adj = col - (0x4B400000u << 7);
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t base = (int64_t)blockIdx.x * blockDim.x; base < Pm.G; base += stride) {
         const int64_t grp = base + threadIdx.x;
@@ -1128,27 +1260,28 @@ __global__ void __launch_bounds__(kThreads) hqq_stream_fixup_kernel(const __grid
         SRow<P> row;
 #pragma unroll
         for (int i = 0; i < P / 2; ++i) row.h[i] = 0;
-        float s = 1.0f, z = 0.0f, lo = 0.0f, hi = 0.0f;
+        SGroup gs;
+        gs.idle();
         if (stale) {
-            load_row<P>(row, Pm.W + grp * P);  // synchronous: the row is read once
-            group_init<NB, P>(row, Pm.eps_tiny, Pm.scale_max, s, z, lo, hi);
+            load_row<P>(row, Pm.W + grp * P, -1);  // synchronous: the row is read once
+            group_init<NB, P>(row, Pm.eps_tiny, Pm.scale_max, gs);
         }
         const int n = stale ? min(b, f) : 0;
         for (int r = 0; __any_sync(kFull, r < n); ++r) {
-#pragma unroll
-            for (int k = 0; k < NQ; ++k) tabw[k * 32 + lane] = __fdiv_rn(__fsub_rn((float)k, z), s);
-            float esum, zsum, maxr;
+            build_table<NQ>(col, gs.s, gs.y, gs.z);
+            float esum, zsum;
             SCodes<NB, P, false> nocodes;
-            stream_round<NB, P, true, false>(row, s, z, tab_adj, esum, zsum, maxr, nocodes);
+            stream_round<NB, P, true, false>(row, gs.s, gs.z, tab_adj, esum, zsum, nocodes);
             const int rr = min(r, K - 1);
-            const bool slow = r < n && maxr > Pm.thr[rr];
-            if (slow) zsum = group_zsum_shrink<NB>(Pm.W + grp * P, P, P, s, z, tab_adj, Pm.beta[rr], Pm.p);
+            const float B = resid_bound(__fadd_rn(gs.lo, gs.z), __fadd_rn(gs.hi, gs.z), gs.A, gs.z, gs.y, kQmax);
+            const bool slow = r < n && B > Pm.thr[rr];
+            if (slow) zsum = group_zsum_shrink<NB>(Pm.W + grp * P, P, P, gs.s, gs.z, tab_adj, Pm.beta[rr], Pm.p);
             const float znew = __fmul_rn(zsum, 1.0f / (float)P);
-            if (r < n) z = znew;
+            if (r < n) gs.z = znew;
         }
         if (stale) {
-            group_store_codes<NB, P>(Pm, row, grp, s, z);
-            write_meta(Pm, grp, s, z, -1);
+            group_store_codes<NB, P>(Pm, row, grp, gs.s, gs.z);
+            stream_meta(Pm, grp, gs.s, gs.y, gs.z, -1);
         }
     }
 }

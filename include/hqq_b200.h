@@ -22,7 +22,8 @@
  *     tail of the last byte or word is zero;
  *   - metadata [HQQ 算法解读, "量化公式：把尺子写出来"]: scale[G] = fp16(1/s) (the page's
  *     Delta) and zero[G] = fp16(z), in group order.
- *   - W must hold finite values.
+ *   - W should hold finite values: a group with a NaN or an infinity gets unspecified codes and
+ *     metadata (the call still completes and touches no memory outside its buffers).
  */
 #ifndef HQQ_B200_H
 #define HQQ_B200_H

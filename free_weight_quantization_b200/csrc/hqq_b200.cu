@@ -854,12 +854,13 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
 // (k - z) * y with y = RN(1/s), refined by two remainder corrections q + RN(a - s q) * y
 // (Markstein, IBM J. Res. Dev. 34(1), 1990: with y = RN(1/s) and q within one ulp of a/s,
 // the correction rounds to RN(a/s)).  The first correction brings the product within one
-// ulp; the second then rounds it.  The quotients must lie in the normal range: with
-// |z| >= 2^-60 (or z = 0), every nonzero |k - z|/s exceeds 2^-80 for s <= 2^15.  Otherwise
-// the lane divides.
+// ulp; the second then rounds it.  The quotients and remainders must stay in the normal
+// range: every nonzero |k - z| is at least min(|z|, 2^-25), so |z| >= 2^-60 (or z = 0) with
+// 2^-60 <= s <= 2^30 keeps each nonzero quotient above 2^-90 and each nonzero remainder
+// above 2^-110.  Outside that the lane divides.
 template <int NQ>
 __device__ __forceinline__ void build_table(uint32_t col, float s, float y, float z) {
-    if (z == 0.0f || fabsf(z) >= 0x1p-60f) {
+    if ((z == 0.0f || fabsf(z) >= 0x1p-60f) && s >= 0x1p-60f && s <= 0x1p30f) {
         const float2 y2 = make_float2(y, y), ns2 = make_float2(-s, -s), nz2 = make_float2(-z, -z);
 #pragma unroll
         for (int k = 0; k < NQ; k += 2) {
@@ -1110,6 +1111,12 @@ __device__ __forceinline__ int64_t claim(const QParams &Pm, bool want) {
     return (want && id < Pm.G) ? id : -1;
 }
 
+// position of the k-th (from 0) set bit of mask, or -1
+__device__ __forceinline__ int nth_set_bit(unsigned mask, int k) {
+    for (int i = 0; i < k; ++i) mask &= mask - 1u;
+    return __ffs(mask) - 1;
+}
+
 template <int NB, int P>
 __global__ void __launch_bounds__(kThreads) hqq_stream_kernel(const __grid_constant__ QParams Pm) {
     extern __shared__ __align__(16) unsigned char smem[];
@@ -1164,6 +1171,32 @@ __global__ void __launch_bounds__(kThreads) hqq_stream_kernel(const __grid_const
             if (need) {
                 nxt = n2;
                 if (nxt >= 0) prefetch_row<P>(slot, Pm.W, nxt, sw);
+            }
+        }
+        // Once nothing is left to claim (a lane whose claim failed holds no group), the k-th
+        // idle lane takes the queued group of the k-th lane that holds one it has not started;
+        // the row is already in that lane's slot.
+        {
+            const unsigned idle_m = __ballot_sync(kFull, cur < 0 && nxt < 0);
+            const unsigned donor_m = __ballot_sync(kFull, cur >= 0 && nxt >= 0);
+            if (idle_m != 0u && donor_m != 0u) {
+                const bool is_donor = (donor_m >> lane) & 1u, is_idle = (idle_m >> lane) & 1u;
+                if (is_donor) prefetch_wait();
+                __syncwarp();
+                const unsigned below = (1u << lane) - 1u;
+                const int npair = min(__popc(idle_m), __popc(donor_m));
+                const int ri = __popc(idle_m & below), rd = __popc(donor_m & below);
+                const bool takes = is_idle && ri < npair;
+                const int src = takes ? nth_set_bit(donor_m, ri) : lane;
+                const int64_t dn = __shfl_sync(kFull, nxt, src);
+                if (takes) {
+                    cur = dn;
+                    load_row<P>(row, slot + (src - lane) * P, slot_swizzle<P>(src));
+                    group_init<NB, P>(row, Pm.eps_tiny, Pm.scale_max, gs);
+                    it = 0;
+                }
+                if (is_donor && rd < npair) nxt = -1;
+                __syncwarp();
             }
         }
         const bool active = cur >= 0;

@@ -25,13 +25,38 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-METRIC = "HQQ quantize+pack Gweights/s at 4096² 4-bit g64; dequant GB/s; % of HBM peak"
+METRIC_ATTN = "HQQ quantize+pack Gweights/s at 4096² 4-bit g64; dequant GB/s; % of HBM peak"
+METRIC = METRIC_ATTN
 UNIT = "Gweights/s"
 ROWS = COLS = 4096
 NBITS, GROUP, AXIS, ITERS = 4, 64, 1, 20
 WORKLOAD = ("0.02*StudentT(4) clipped to +-1, fp16 4096x4096 (attention-projection-shaped), seed 1; "
             "4-bit, group 64, axis 1, <=20 rounds, p=0.7, beta=10, kappa=1.01")
 ROTATE = 8
+CASE = None                  # the workloads.Case being timed (set by select())
+GEN_DESC = {"outlier_normal": "N(0, 0.02^2) with 0.1% of entries replaced by +-U(0.2, 1.0)",
+            "student_t": "0.02*StudentT(4) clipped to +-1",
+            "row_lognormal": "N(0, 0.015^2) x per-row LogNormal(0, 0.3)"}
+SINGLE = {"small": "SMALL", "attn": "ATTN", "mlp_b2": "MLP_B2", "mlp_b3": "MLP_B3", "attn_ax0": "ATTN_AX0"}
+
+
+def select(name: str):
+    """Point the module's workload constants at one of the single-matrix configurations."""
+    global CASE, ROWS, COLS, NBITS, GROUP, AXIS, WORKLOAD, ROTATE, METRIC
+    from free_weight_quantization_b200 import workloads as wl
+    c = getattr(wl, SINGLE[name])
+    CASE = c
+    ROWS, COLS, NBITS, GROUP, AXIS = c.rows, c.cols, c.nbits, c.group_size, c.axis
+    WORKLOAD = (f"{GEN_DESC[c.gen]}, fp16 {c.rows}x{c.cols}, seed {c.seed}; {c.nbits}-bit, "
+                f"group {c.group_size}, axis {c.axis}, <=20 rounds, p=0.7, beta=10, kappa=1.01")
+    if name == "attn":
+        METRIC = METRIC_ATTN
+        WORKLOAD = ("0.02*StudentT(4) clipped to +-1, fp16 4096x4096 (attention-projection-shaped), "
+                    "seed 1; 4-bit, group 64, axis 1, <=20 rounds, p=0.7, beta=10, kappa=1.01")
+    else:
+        METRIC = f"HQQ quantize+pack Gweights/s at {c.rows}x{c.cols} {c.nbits}-bit g{c.group_size} axis {c.axis}; dequant GB/s; % of HBM peak"
+    # enough rotating copies that the inputs outgrow twice the 126 MB L2
+    ROTATE = max(8, -(-252_000_000 // (2 * c.rows * c.cols)))
 ISSUE_LANES_PER_SM = 128     # 4 SM sub-partitions x 32 lanes issue one instruction per clock
 ALU_OPS_INIT, ALU_OPS_ROUND, ALU_OPS_FINAL = 3, 12, 6   # algorithmic ops per weight
 
@@ -146,11 +171,12 @@ def run_reference(args, ws, rank):
     import oracle
     from free_weight_quantization_b200 import workloads as wl
     oracle.build()
-    W = wl.ATTN.make()
-    rows = 256                        # each step: a 256 x 4096 slice (1 M weights)
+    W = CASE.make()
+    rows = min(256, ROWS)             # each step: a slice of up to 256 rows of the matrix
     times = []
     for i in range(args.warmup + args.steps):
-        sl = np.ascontiguousarray(W[(i % 16) * rows:(i % 16 + 1) * rows])
+        nsl = ROWS // rows
+        sl = np.ascontiguousarray(W[(i % nsl) * rows:(i % nsl + 1) * rows])
         t0 = time.perf_counter()
         r = oracle.quantize(sl, NBITS, GROUP, AXIS, iters=ITERS)
         oracle.dequant(r["packed"], r["scale"], r["zero"], rows, COLS, NBITS, GROUP, AXIS)
@@ -159,7 +185,8 @@ def run_reference(args, ws, rank):
             times.append(dt)
     n = rows * COLS
     value = n * len(times) / sum(times) / 1e9
-    sample = f"{args.steps} slices of 256x4096 rows of the 4096x4096 workload, quantize+pack+dequant"
+    sample = (f"{args.steps} slices of {rows}x{COLS} of the {ROWS}x{COLS} workload, "
+              "quantize+pack+dequant")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
@@ -172,33 +199,155 @@ def run_reference(args, ws, rank):
 
 
 def cpu_baseline():
-    """The oracle timed once on the full 4096x4096 matrix (about 15 s on one core)."""
+    """The oracle timed on the full matrix of the workload, repeated until about 3 s have
+    passed (one pass of a 4096x4096 matrix takes about 9 s on one core)."""
     import oracle
-    from free_weight_quantization_b200 import workloads as wl
     oracle.build()
-    W = wl.ATTN.make()
-    t0 = time.perf_counter()
-    r = oracle.quantize(W, NBITS, GROUP, AXIS, iters=ITERS)
-    oracle.dequant(r["packed"], r["scale"], r["zero"], ROWS, COLS, NBITS, GROUP, AXIS)
-    dt = time.perf_counter() - t0
-    return {"value": ROWS * COLS / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": "one 4096x4096 matrix of the workload, quantize+pack+dequant, "
-                      f"{dt:.1f} s single-threaded"}
+    W = CASE.make()
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        r = oracle.quantize(W, NBITS, GROUP, AXIS, iters=ITERS)
+        oracle.dequant(r["packed"], r["scale"], r["zero"], ROWS, COLS, NBITS, GROUP, AXIS)
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= 3.0:
+            break
+    return {"value": reps * ROWS * COLS / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{reps} pass(es) over the {ROWS}x{COLS} matrix of the workload, "
+                      f"quantize+pack+dequant, {dt:.1f} s single-threaded"}
+
+
+STACK_WORKLOAD = ("synthetic 7B-like stack: 32 layers x (4 x 4096x4096 + 3 x 4096x11008) fp16, "
+                  "0.02*StudentT(4) clipped to +-1 drawn on the GPU from per-matrix seeds; 4-bit, "
+                  "group 64, axis 1, per-tensor early stop; quantize all then dequantize all")
+
+
+def run_stack(args, ws, rank, local):
+    """One step = quantize+pack every matrix of the stack, then dequantize every matrix.
+    Under torchrun the 224 matrices are split across ranks (no communication: strong scaling)."""
+    import torch
+    import torch.distributed as dist
+
+    from free_weight_quantization_b200 import hqq
+    from free_weight_quantization_b200 import workloads as wl
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        dist.init_process_group("nccl", device_id=dev,
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    keys = [(l, i) for l in range(wl.STACK_LAYERS) for i in range(len(wl.STACK_SHAPES))]
+    mine = keys[rank::ws]
+    Ws = [wl.stack_matrix_torch(l, i, dev) for l, i in mine]
+    outs = [hqq.hqq_quantize(W, NBITS, GROUP, AXIS, iters=ITERS, debug=True) for W in Ws]
+    torch.cuda.synchronize()
+    rounds = sum(int(q.rounds.to(torch.int64).sum().item()) for q in outs)
+    iters = [int(q.iters_run.item()) for q in outs]
+    for q in outs:
+        q.iters_run = q.s = q.z = q.err_trace = q.rounds = None
+    deqs = [torch.empty_like(W) for W in Ws]
+    work = {}
+    for W in Ws:
+        r, c = W.shape
+        if (r, c) not in work:
+            work[(r, c)] = torch.empty(max(16, hqq.hqq_quantize_workspace_bytes(r, c, NBITS, GROUP, AXIS, ITERS)),
+                                       dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        for W, q in zip(Ws, outs):
+            hqq.hqq_quantize(W, NBITS, GROUP, AXIS, iters=ITERS, out=q, workspace=work[tuple(W.shape)])
+        for q, d in zip(outs, deqs):
+            hqq.hqq_dequantize(q, out=d)
+
+    for _ in range(args.warmup):
+        step()
+    sampler = ClockSampler(local).start()
+    time.sleep(0.3)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    tw0 = time.time()
+    a.record(stream)
+    for _ in range(args.steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    tw1 = time.time()
+    if ws > 1:
+        dist.barrier()
+    ms = a.elapsed_time(b) / args.steps
+    sampler.stop()
+    clocks = sampler.summary(tw0, tw1)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if ws > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = t.item()
+    n_all = sum(r * c for r, c in (wl.STACK_SHAPES[i] for _, i in keys))
+    n_mine = sum(W.numel() for W in Ws)
+    if rank == 0:
+        pk = peaks()
+        alu_peak = 148 * ISSUE_LANES_PER_SM * pk["sm_max_mhz"] * 1e6 / 1e12
+        alg_ops = n_mine * (ALU_OPS_INIT + ALU_OPS_FINAL) + GROUP * rounds * ALU_OPS_ROUND
+        ach = alg_ops / (ms / 1e3) / 1e12 * ws
+        line = {
+            "metric": METRIC, "value": n_all / (ms / 1e3) / 1e9, "unit": UNIT, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": STACK_WORKLOAD, "matrices": len(keys), "weights": n_all,
+                       "iters_run_min_max": [min(iters), max(iters)],
+                       "l2": "inputs larger than L2 (12.95 GB stack)",
+                       "parallelism": f"matrices split across {ws} rank(s)"},
+            "roofline": {"bound": "alu", "kernel": "hqq_quantize + hqq_dequantize over the stack",
+                         "achieved": ach, "peak": alu_peak, "unit": "Tops/s", "frac": ach / alu_peak,
+                         "traffic": None, "alg_ops_per_step": alg_ops * ws},
+            "e2e": None,
+            "gpu_launches": 3 * len(Ws) * args.steps,
+            "clocks": clocks,
+        }
+        if not args.no_cpu_baseline:
+            Wh = Ws[0].cpu().numpy()
+            import oracle
+            oracle.build()
+            t0 = time.perf_counter()
+            r = oracle.quantize(Wh, NBITS, GROUP, AXIS, iters=ITERS)
+            oracle.dequant(r["packed"], r["scale"], r["zero"], Wh.shape[0], Wh.shape[1], NBITS, GROUP, AXIS)
+            dt = time.perf_counter() - t0
+            line["cpu_baseline"] = {"value": Wh.size / dt / 1e9, "unit": UNIT, "cores": 1,
+                                    "kind": "oracle",
+                                    "sample": f"layer 0 matrix 0 (4096x4096) of the stack, {dt:.1f} s "
+                                              "single-threaded; the stack is 247x its size"}
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.destroy_process_group()
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5000)
+    ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
+    ap.add_argument("--workload", default="attn", choices=list(SINGLE) + ["stack"],
+                    help="attn: the 4096x4096 headline matrix (default); small, mlp_b2, mlp_b3, "
+                         "attn_ax0: the other single-matrix configurations; stack: the 7B-like "
+                         "224-matrix stack")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.steps is None:
+        args.steps = {"attn": 5000, "small": 20000, "attn_ax0": 3000, "stack": 20}.get(args.workload, 1500)
+    if args.workload != "stack":
+        select(args.workload)
     ws, rank, local = dist_setup()
 
     if args.impl == "reference":
         run_reference(args, ws, rank)
+        return
+    if args.workload == "stack":
+        run_stack(args, ws, rank, local)
         return
 
     import torch
@@ -216,7 +365,7 @@ def main():
                                 timeout=__import__("datetime").timedelta(seconds=120))
 
     # every rank quantizes its own copies of the workload matrix
-    W0 = torch.from_numpy(wl.ATTN.make())
+    W0 = torch.from_numpy(CASE.make())
     Ws = [W0.to(dev) for _ in range(ROTATE)]
     N = ROWS * COLS
     G = N // GROUP
@@ -260,6 +409,18 @@ def main():
     q_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
     d_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
 
+    # dequantize alone, back to back over the rotating buffers: its sustained throughput, without
+    # the per-call event brackets of the step loop (each adds about as much as a short launch)
+    nb2b = max(2 * ROTATE, min(args.steps, 400))
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    b0.record(stream)
+    for i in range(nb2b):
+        hqq.hqq_dequantize(outs[i % ROTATE], out=deqs[i % ROTATE])
+    b1.record(stream)
+    torch.cuda.synchronize()
+    d_b2b_ms = b0.elapsed_time(b1) / nb2b
+
     # end to end through the public API: pinned host W in, packed codes + metadata + dequantized
     # W out, copies inside the timed region
     Wh = W0.pin_memory()
@@ -293,10 +454,10 @@ def main():
     clocks = sampler.summary(tw0, tw1)
 
     # max over ranks
-    t = torch.tensor([total_ms, q_ms, d_ms, e2e_ms], dtype=torch.float64, device=dev)
+    t = torch.tensor([total_ms, q_ms, d_ms, e2e_ms, d_b2b_ms], dtype=torch.float64, device=dev)
     if ws > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, q_ms, d_ms, e2e_ms = t.tolist()
+    total_ms, q_ms, d_ms, e2e_ms, d_b2b_ms = t.tolist()
 
     if rank == 0:
         pk = peaks()
@@ -314,9 +475,12 @@ def main():
         if rounds is not None:
             alg_ops = N * (ALU_OPS_INIT + ALU_OPS_FINAL) + GROUP * rounds * ALU_OPS_ROUND
             ach = alg_ops / q_s / 1e12
-            roofline = {"bound": "alu", "kernel": "hqq_quantize (hqq_stream_kernel + hqq_stream_fixup_kernel)",
+            stream = AXIS == 1 and NBITS != 3 and GROUP in (16, 32, 64, 128) and GROUP * NBITS % 32 == 0
+            kname = ("hqq_quantize (hqq_stream_kernel + hqq_stream_fixup_kernel)" if stream else
+                     "hqq_quantize (hqq_search_kernel + hqq_fixup_kernel)")
+            roofline = {"bound": "alu", "kernel": kname,
                         "achieved": ach, "peak": alu_peak, "unit": "Tops/s", "frac": ach / alu_peak,
-                        "traffic": profiled_traffic(),
+                        "traffic": profiled_traffic() if CASE.name.startswith("student-t 4096x4096 b4 g64") else None,
                         "peak_src": f"148 SMs x 128 lanes x {pk['sm_max_mhz']:.0f} MHz (max clock)",
                         "alg_ops_per_launch": alg_ops, "group_rounds": rounds}
         line = {
@@ -332,6 +496,9 @@ def main():
             "quant_us": q_s * 1e6, "dequant_us": d_s * 1e6,
             "quant_hbm_gbs": hbm_q, "quant_hbm_frac": hbm_q / pk["hbm_gbs"],
             "dequant_gbs": hbm_d, "dequant_hbm_frac": hbm_d / pk["hbm_gbs"],
+            "dequant_back_to_back": {"us": d_b2b_ms * 1e3, "gbs": alg_bytes / (d_b2b_ms / 1e3) / 1e9,
+                                     "hbm_frac": alg_bytes / (d_b2b_ms / 1e3) / 1e9 / pk["hbm_gbs"],
+                                     "launches": nb2b},
             "hbm_peak_gbs": pk["hbm_gbs"], "hbm_peak_src": pk["src"],
             "alg_bytes_per_launch": alg_bytes,
             "roofline": roofline,

@@ -56,6 +56,7 @@ struct QParams {
     int K;          // iteration cap
     int stride;     // floats per group row of the shared tile
     int tile;       // groups per tile
+    int stream_warps;  // warps of each streaming-engine CTA that take groups (the rest idle)
     uint8_t *packed;
     int64_t packed_bytes;
     __half *scale, *zero;
@@ -1118,7 +1119,7 @@ __device__ __forceinline__ int nth_set_bit(unsigned mask, int k) {
 }
 
 template <int NB, int P>
-__global__ void __launch_bounds__(kThreads) hqq_stream_kernel(const __grid_constant__ QParams Pm) {
+__global__ void __launch_bounds__(kThreads, P <= 64 ? 2 : 1) hqq_stream_kernel(const __grid_constant__ QParams Pm) {
     extern __shared__ __align__(16) unsigned char smem[];
     constexpr int NQ = 1 << NB;
     constexpr float kQmax = (float)(NQ - 1);
@@ -1154,7 +1155,9 @@ __global__ void __launch_bounds__(kThreads) hqq_stream_kernel(const __grid_const
     gs.idle();
     int it = 0;
     int64_t cur = -1;
-    int64_t nxt = claim(Pm, true);
+    // a small tensor is spread thin: only the first stream_warps warps of each CTA take groups,
+    // so its few groups run on many SMs rather than crowding a few
+    int64_t nxt = warp < Pm.stream_warps ? claim(Pm, true) : -1;
     if (nxt >= 0) prefetch_row<P>(slot, Pm.W, nxt, sw);
     while (true) {
         // ---- a lane without a group takes the prefetched one and prefetches another
@@ -1284,37 +1287,54 @@ __global__ void __launch_bounds__(kThreads) hqq_stream_fixup_kernel(const __grid
     float *tabw = reinterpret_cast<float *>(smem) + warp * NQ * 32;
     const uint32_t col = (uint32_t)__cvta_generic_to_shared(tabw + lane);
     const uint32_t tab_adj = col - (0x4B400000u << 7);
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t base = (int64_t)blockIdx.x * blockDim.x; base < Pm.G; base += stride) {
-        const int64_t grp = base + threadIdx.x;
-        const int f = grp < Pm.G ? (int)__ldcg(Pm.fk + grp) : 0;
-        const bool stale = grp < Pm.G && f > b;
-        if (!__any_sync(kFull, stale)) continue;
-        SRow<P> row;
+    // each lane scans 16 groups' last rounds with one 16-byte load (fk is 16-byte aligned: it
+    // follows the 32-byte-multiple round sums in the workspace), then the warp replays the
+    // stale ones, one per lane at a time
+    const int64_t wstride = (int64_t)gridDim.x * kWarps * 512;
+    for (int64_t wbase = ((int64_t)blockIdx.x * kWarps + warp) * 512; wbase < Pm.G; wbase += wstride) {
+        const int64_t c0 = wbase + 16 * lane;
+        uint32_t mask = 0;  // bit j: group c0 + j is stale
+        if (c0 + 16 <= Pm.G) {
+            const uint4 v = __ldcg(reinterpret_cast<const uint4 *>(Pm.fk + c0));
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int i = 0; i < P / 2; ++i) row.h[i] = 0;
-        SGroup gs;
-        gs.idle();
-        if (stale) {
-            load_row<P>(row, Pm.W + grp * P, -1);  // synchronous: the row is read once
-            group_init<NB, P>(row, Pm.eps_tiny, Pm.scale_max, gs);
+            for (int j = 0; j < 16; ++j)
+                if ((int)((w4[j >> 2] >> (8 * (j & 3))) & 0xffu) > b) mask |= 1u << j;
+        } else {
+            for (int j = 0; j < 16 && c0 + j < Pm.G; ++j)
+                if ((int)__ldcg(Pm.fk + c0 + j) > b) mask |= 1u << j;
         }
-        const int n = stale ? min(b, f) : 0;
-        for (int r = 0; __any_sync(kFull, r < n); ++r) {
-            build_table<NQ>(col, gs.s, gs.y, gs.z);
-            float esum, zsum;
-            SCodes<NB, P, false> nocodes;
-            stream_round<NB, P, true, false>(row, gs.s, gs.z, tab_adj, esum, zsum, nocodes);
-            const int rr = min(r, K - 1);
-            const float B = resid_bound(__fadd_rn(gs.lo, gs.z), __fadd_rn(gs.hi, gs.z), gs.A, gs.z, gs.y, kQmax);
-            const bool slow = r < n && B > Pm.thr[rr];
-            if (slow) zsum = group_zsum_shrink<NB>(Pm.W + grp * P, P, P, gs.s, gs.z, tab_adj, Pm.beta[rr], Pm.p);
-            const float znew = __fmul_rn(zsum, 1.0f / (float)P);
-            if (r < n) gs.z = znew;
-        }
-        if (stale) {
-            group_store_codes<NB, P>(Pm, row, grp, gs.s, gs.z);
-            stream_meta(Pm, grp, gs.s, gs.y, gs.z, -1);
+        while (__any_sync(kFull, mask != 0u)) {
+            const bool stale = mask != 0u;
+            const int64_t grp = stale ? c0 + (__ffs(mask) - 1) : 0;
+            mask &= mask - 1u;
+            const int f = stale ? (int)__ldcg(Pm.fk + grp) : 0;
+            SRow<P> row;
+#pragma unroll
+            for (int i = 0; i < P / 2; ++i) row.h[i] = 0;
+            SGroup gs;
+            gs.idle();
+            if (stale) {
+                load_row<P>(row, Pm.W + grp * P, -1);  // synchronous: the row is read once
+                group_init<NB, P>(row, Pm.eps_tiny, Pm.scale_max, gs);
+            }
+            const int n = stale ? min(b, f) : 0;
+            for (int r = 0; __any_sync(kFull, r < n); ++r) {
+                build_table<NQ>(col, gs.s, gs.y, gs.z);
+                float esum, zsum;
+                SCodes<NB, P, false> nocodes;
+                stream_round<NB, P, true, false>(row, gs.s, gs.z, tab_adj, esum, zsum, nocodes);
+                const int rr = min(r, K - 1);
+                const float B = resid_bound(__fadd_rn(gs.lo, gs.z), __fadd_rn(gs.hi, gs.z), gs.A, gs.z, gs.y, kQmax);
+                const bool slow = r < n && B > Pm.thr[rr];
+                if (slow) zsum = group_zsum_shrink<NB>(Pm.W + grp * P, P, P, gs.s, gs.z, tab_adj, Pm.beta[rr], Pm.p);
+                const float znew = __fmul_rn(zsum, 1.0f / (float)P);
+                if (r < n) gs.z = znew;
+            }
+            if (stale) {
+                group_store_codes<NB, P>(Pm, row, grp, gs.s, gs.z);
+                stream_meta(Pm, grp, gs.s, gs.y, gs.z, -1);
+            }
         }
     }
 }
@@ -1604,13 +1624,17 @@ cudaError_t launch_stream(const QParams &Pm, cudaStream_t st) {
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k1, kThreads, smem) != cudaSuccess ||
         per_sm < 1)
         per_sm = 1;
-    const int64_t lanes_needed = (Pm.G + 31) / 32 * 32;
+    // warps that take groups in each CTA: all of them once the tensor fills the resident grid,
+    // fewer (down to one) for a small tensor, so that its groups land on as many SMs as possible
+    const int64_t slots = (int64_t)sms * per_sm;
+    const int64_t warps_needed = (Pm.G + 31) / 32;
+    QParams Q = Pm;
+    Q.stream_warps = (int)std::min<int64_t>(kWarps, std::max<int64_t>(1, (warps_needed + slots - 1) / slots));
     const unsigned blocks = (unsigned)std::max<int64_t>(
-        1, std::min<int64_t>((int64_t)sms * per_sm, (lanes_needed + kThreads - 1) / kThreads));
-    k1<<<blocks, kThreads, smem, st>>>(Pm);
-    const unsigned fix_blocks = (unsigned)std::min<int64_t>((int64_t)sms * per_sm,
-                                                            (Pm.G + kThreads - 1) / kThreads);
-    k2<<<std::max(1u, fix_blocks), kThreads, smem, st>>>(Pm);
+        1, std::min<int64_t>(slots, (warps_needed + Q.stream_warps - 1) / Q.stream_warps));
+    k1<<<blocks, kThreads, smem, st>>>(Q);
+    const unsigned fix_blocks = (unsigned)std::min<int64_t>(slots, (Pm.G + kWarps * 512 - 1) / (kWarps * 512));
+    k2<<<std::max(1u, fix_blocks), kThreads, smem, st>>>(Q);
     return cudaGetLastError();
 }
 

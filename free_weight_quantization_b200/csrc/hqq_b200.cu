@@ -57,6 +57,7 @@ struct QParams {
     int stride;     // floats per group row of the shared tile
     int tile;       // groups per tile
     int stream_warps;  // warps of each streaming-engine CTA that take groups (the rest idle)
+    int64_t acc_words; // 64-bit words of round sums and control words zeroed before each call
     uint8_t *packed;
     int64_t packed_bytes;
     __half *scale, *zero;
@@ -635,6 +636,19 @@ struct Ctl {
     unsigned long long pad;
 };
 
+// Programmatic dependent launch: a kernel launched with programmatic stream serialization may
+// become resident while its predecessor still runs; wait_prerequisite() returns once the
+// predecessor grid has completed and its writes are visible, and allow_dependents() lets the
+// next grid be scheduled once every CTA of this one has called it (or exited).
+__device__ __forceinline__ void wait_prerequisite() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// zeroes the per-call round sums and control words of the workspace (n 64-bit words)
+__global__ void __launch_bounds__(256) hqq_zero_kernel(u64 *acc, int n) {
+    allow_dependents();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) acc[i] = 0ull;
+}
+
 __device__ __forceinline__ Ctl *ctl_of(const QParams &P) {
     return reinterpret_cast<Ctl *>(P.acc + 4 * (P.K > 0 ? P.K : 1));
 }
@@ -703,6 +717,9 @@ __global__ void __launch_bounds__(kThreads, 2) hqq_search_kernel(const __grid_co
     int mf = 0;
     for (int i = threadIdx.x; i < tg; i += kThreads) mf = max(mf, DIRECT ? (int)__ldcg(P.fk + t0 + i) : (int)S.f_t[i]);
     atomicMax(&maxf, mf);
+    // the global round sums were zeroed by the kernel launched before this one
+    wait_prerequisite();
+    allow_dependents();
     // this tile's per-round sums (16-bit chunks) -> 128-bit global sums
     for (int i = threadIdx.x; i < 2 * K; i += kThreads) {
         unsigned __int128 v = 0;
@@ -741,6 +758,8 @@ __global__ void __launch_bounds__(kThreads, 2) hqq_search_kernel(const __grid_co
 template <int NB, int L, bool FULL, bool DIRECT>
 __global__ void __launch_bounds__(kThreads, 2) hqq_fixup_kernel(const __grid_constant__ QParams P) {
     extern __shared__ __align__(16) unsigned char smem[];
+    wait_prerequisite();  // the search kernel has finished and listed the stale tiles
+    allow_dependents();
     Ctl *c = ctl_of(P);
     const int nstale = __ldcg(&c->nstale);
     if ((int)blockIdx.x >= nstale) return;
@@ -1155,6 +1174,8 @@ __global__ void __launch_bounds__(kThreads, P <= 64 ? 2 : 1) hqq_stream_kernel(c
     gs.idle();
     int it = 0;
     int64_t cur = -1;
+    // the round sums and the group counter were zeroed by the kernel launched before this one
+    wait_prerequisite();
     // a small tensor is spread thin: only the first stream_warps warps of each CTA take groups,
     // so its few groups run on many SMs rather than crowding a few
     int64_t nxt = warp < Pm.stream_warps ? claim(Pm, true) : -1;
@@ -1249,6 +1270,7 @@ __global__ void __launch_bounds__(kThreads, P <= 64 ? 2 : 1) hqq_stream_kernel(c
             cur = -1;
         }
     }
+    allow_dependents();  // the fixup kernel may take the SMs this CTA leaves
     // this warp's per-round sums (16-bit chunks) -> 128-bit global sums
     __syncwarp();
     for (int i = lane; i < 2 * K; i += 32) {
@@ -1281,6 +1303,7 @@ __global__ void __launch_bounds__(kThreads) hqq_stream_fixup_kernel(const __grid
     constexpr int NQ = 1 << NB;
     constexpr float kQmax = (float)(NQ - 1);
     const int K = Pm.K;
+    wait_prerequisite();  // the stream kernel has finished and applied the stop rule
     const int b = __ldcg(&ctl_of(Pm)->b);
     if (K == 0 || b >= K - 1) return;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -1344,6 +1367,7 @@ template <int NB>
 __global__ void pack_codes_kernel(const uint8_t *codes, int64_t N, uint8_t *packed,
                                   int64_t packed_bytes) {
     constexpr int CPW = Pack<NB>::cpw;
+    wait_prerequisite();  // the fixup kernel has rewritten its stale codes
     const int64_t nw = (N + CPW - 1) / CPW;
     for (int64_t wi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; wi < nw;
          wi += (int64_t)gridDim.x * blockDim.x) {
@@ -1578,6 +1602,24 @@ int make_plan(int64_t rows, int64_t cols, int nbits, int64_t group_size, int axi
 bool aligned_to(const void *p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
 
 
+// launches kernel<<<grid, block, smem, st>>>(args...) with programmatic stream serialization:
+// the launch overlaps the kernel before it, which the kernel waits for in wait_prerequisite()
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, int smem,
+                       cudaStream_t st, Args... args) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 template <int NB, int L, bool FULL, bool DIRECT>
 cudaError_t launch_quant(const QParams &P, int64_t ntiles, cudaStream_t st) {
     const SmemLayout lay = smem_layout(P.tile, P.stride, 1 << NB, L, P.K);
@@ -1587,13 +1629,19 @@ cudaError_t launch_quant(const QParams &P, int64_t ntiles, cudaStream_t st) {
     e = cudaFuncSetAttribute(hqq_fixup_kernel<NB, L, FULL, DIRECT>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total);
     if (e != cudaSuccess) return e;
-    hqq_search_kernel<NB, L, FULL, DIRECT><<<(unsigned)ntiles, kThreads, lay.total, st>>>(P);
+    // zero kernel -> search -> fixup (-> pack), the later ones with programmatic launches
+    hqq_zero_kernel<<<1, 256, 0, st>>>(P.acc, (int)P.acc_words);
+    e = launch_pdl(hqq_search_kernel<NB, L, FULL, DIRECT>, (unsigned)ntiles, kThreads, lay.total, st, P);
+    if (e != cudaSuccess) return e;
     const unsigned fix_blocks = (unsigned)std::min<int64_t>(ntiles, 148 * 2);  // one wave
-    hqq_fixup_kernel<NB, L, FULL, DIRECT><<<fix_blocks, kThreads, lay.total, st>>>(P);
+    e = launch_pdl(hqq_fixup_kernel<NB, L, FULL, DIRECT>, fix_blocks, kThreads, lay.total, st, P);
+    if (e != cudaSuccess) return e;
     if (P.codes_u8) {
         const int64_t nw = (P.N + Pack<NB>::cpw - 1) / Pack<NB>::cpw;
         const unsigned blocks = (unsigned)std::min<int64_t>((nw + 255) / 256, 148 * 16);
-        pack_codes_kernel<NB><<<blocks, 256, 0, st>>>(P.codes_u8, P.N, P.packed, P.packed_bytes);
+        e = launch_pdl(pack_codes_kernel<NB>, blocks, 256, 0, st, (const uint8_t *)P.codes_u8, P.N,
+                       P.packed, P.packed_bytes);
+        if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
 }
@@ -1632,9 +1680,14 @@ cudaError_t launch_stream(const QParams &Pm, cudaStream_t st) {
     Q.stream_warps = (int)std::min<int64_t>(kWarps, std::max<int64_t>(1, (warps_needed + slots - 1) / slots));
     const unsigned blocks = (unsigned)std::max<int64_t>(
         1, std::min<int64_t>(slots, (warps_needed + Q.stream_warps - 1) / Q.stream_warps));
-    k1<<<blocks, kThreads, smem, st>>>(Q);
+    // zero kernel -> stream kernel -> fixup kernel, each later one launched with programmatic
+    // stream serialization so that its launch overlaps the kernel before it
+    hqq_zero_kernel<<<1, 256, 0, st>>>(Pm.acc, (int)Pm.acc_words);
+    e = launch_pdl(k1, blocks, kThreads, smem, st, Q);
+    if (e != cudaSuccess) return e;
     const unsigned fix_blocks = (unsigned)std::min<int64_t>(slots, (Pm.G + kWarps * 512 - 1) / (kWarps * 512));
-    k2<<<std::max(1u, fix_blocks), kThreads, smem, st>>>(Q);
+    e = launch_pdl(k2, std::max(1u, fix_blocks), kThreads, smem, st, Q);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -1752,9 +1805,9 @@ extern "C" int hqq_quantize(const void *W, int64_t rows, int64_t cols, int nbits
         beta = beta * o.kappa;
     }
     cudaStream_t st = (cudaStream_t)stream;
-    if (cudaMemsetAsync(workspace, 0, pl.ws_acc, st) != cudaSuccess) return HQQ_ERR_CUDA;
+    P.acc_words = (int64_t)(pl.ws_acc / sizeof(u64));
     cudaError_t e;
-    if (pl.stream) {  // one lane per group
+    if (pl.stream) {  // one lane per group (each launcher zeroes the round sums itself)
         e = nbits == 4 ? launch_stream_nb<4>(P, pl.P, st) : launch_stream_nb<2>(P, pl.P, st);
     } else {
         const bool direct = axis == 1 && pl.g % 16 == 0;

@@ -1407,6 +1407,8 @@ __global__ void __launch_bounds__(kDqThreads) hqq_dequant_kernel(
     constexpr uint32_t MASK = (1u << NB) - 1u;
     const int64_t nwords = (N + CPW - 1) / CPW;
     const int64_t wbase = (int64_t)blockIdx.x * (kDqThreads * kDqU) + threadIdx.x;
+    wait_prerequisite();  // the codes may come from the kernel launched just before
+    allow_dependents();
     uint32_t wd[kDqU];
 #pragma unroll
     for (int u = 0; u < kDqU; ++u) {
@@ -1507,8 +1509,26 @@ __global__ void __launch_bounds__(kDqThreads) hqq_dequant_kernel(
     }
 }
 
+// launches kernel<<<grid, block, smem, st>>>(args...) with programmatic stream serialization:
+// the launch overlaps the kernel before it, which the kernel waits for in wait_prerequisite()
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, int smem,
+                       cudaStream_t st, Args... args) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 template <int NB>
-void launch_dequant(const uint8_t *pk, const __half *sc, const __half *ze, int64_t N, int g,
+cudaError_t launch_dequant(const uint8_t *pk, const __half *sc, const __half *ze, int64_t N, int g,
                     int64_t G, int axis, int64_t pb, __half *out, cudaStream_t st) {
     constexpr int CPW = Pack<NB>::cpw;
     const int64_t nwords = (N + CPW - 1) / CPW;
@@ -1520,12 +1540,12 @@ void launch_dequant(const uint8_t *pk, const __half *sc, const __half *ze, int64
         if ((wpg & (wpg - 1)) == 0) { shift = 0; while ((1 << shift) < wpg) ++shift; }
     }
     const bool vec_meta = CPW % 8 == 0 && G % 8 == 0 && (((uintptr_t)sc | (uintptr_t)ze) & 15) == 0;
+    // programmatic launch: overlaps the kernel before it, which the kernel waits for
     if (axis == 1 && g % CPW == 0)
-        hqq_dequant_kernel<NB, 0><<<blocks, kDqThreads, 0, st>>>(pw, sc, ze, N, g, G, pb, shift, false, out);
-    else if (axis == 1)
-        hqq_dequant_kernel<NB, 1><<<blocks, kDqThreads, 0, st>>>(pw, sc, ze, N, g, G, pb, -1, false, out);
-    else
-        hqq_dequant_kernel<NB, 2><<<blocks, kDqThreads, 0, st>>>(pw, sc, ze, N, g, G, pb, -1, vec_meta, out);
+        return launch_pdl(hqq_dequant_kernel<NB, 0>, blocks, kDqThreads, 0, st, pw, sc, ze, N, g, G, pb, shift, false, out);
+    if (axis == 1)
+        return launch_pdl(hqq_dequant_kernel<NB, 1>, blocks, kDqThreads, 0, st, pw, sc, ze, N, g, G, pb, -1, false, out);
+    return launch_pdl(hqq_dequant_kernel<NB, 2>, blocks, kDqThreads, 0, st, pw, sc, ze, N, g, G, pb, -1, vec_meta, out);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1601,24 +1621,6 @@ int make_plan(int64_t rows, int64_t cols, int nbits, int64_t group_size, int axi
 
 bool aligned_to(const void *p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
 
-
-// launches kernel<<<grid, block, smem, st>>>(args...) with programmatic stream serialization:
-// the launch overlaps the kernel before it, which the kernel waits for in wait_prerequisite()
-template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, int smem,
-                       cudaStream_t st, Args... args) {
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(block);
-    cfg.dynamicSmemBytes = (size_t)smem;
-    cfg.stream = st;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, args...);
-}
 
 template <int NB, int L, bool FULL, bool DIRECT>
 cudaError_t launch_quant(const QParams &P, int64_t ntiles, cudaStream_t st) {
@@ -1835,12 +1837,13 @@ extern "C" int hqq_dequantize(const void *packed, const void *scale, const void 
     const uint8_t *pk = (const uint8_t *)packed;
     const __half *sc = (const __half *)scale, *ze = (const __half *)zero;
     __half *out = (__half *)W_out;
+    cudaError_t e;
     switch (nbits) {
-    case 4: launch_dequant<4>(pk, sc, ze, pl.N, pl.g, pl.G, axis, pb, out, st); break;
-    case 3: launch_dequant<3>(pk, sc, ze, pl.N, pl.g, pl.G, axis, pb, out, st); break;
-    default: launch_dequant<2>(pk, sc, ze, pl.N, pl.g, pl.G, axis, pb, out, st); break;
+    case 4: e = launch_dequant<4>(pk, sc, ze, pl.N, pl.g, pl.G, axis, pb, out, st); break;
+    case 3: e = launch_dequant<3>(pk, sc, ze, pl.N, pl.g, pl.G, axis, pb, out, st); break;
+    default: e = launch_dequant<2>(pk, sc, ze, pl.N, pl.g, pl.G, axis, pb, out, st); break;
     }
-    return cudaGetLastError() == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
+    return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
 }
 
 extern "C" const char *hqq_strerror(int code) {

@@ -1137,6 +1137,217 @@ __device__ __forceinline__ int nth_set_bit(unsigned mask, int k) {
     return __ffs(mask) - 1;
 }
 
+// ------------------------------------------------------------------------------------------
+// Tail of the streaming engine.  Once the global counter is exhausted, a warp whose lanes are
+// mostly idle would spend full rounds on its last few groups, and these few long chains set
+// the kernel's end.  The warp then re-splits its remaining groups over L lanes each (2 to
+// 16): lane l of a segment holds elements [l E, (l+1) E) of the group (E = P/L, whole 32-bit
+// words of codes), builds every L-th table entry, and the segment adds its partial sums with
+// xor shuffles.  Each lane's chunks are summed by recursive halving and the shuffle levels
+// continue the halving across lanes, so the group sums keep the oracle's order.  As groups
+// finish, the warp splits again into wider segments.
+// The split costs about twice the instructions per group-round, so it only pays once the
+// warp is nearly empty: at most kTailLanes groups left (4096^2 4-bit g64: 103.7 -> 97.8 us
+// with 4; a threshold of 16 was slower than no split at all).
+// ------------------------------------------------------------------------------------------
+constexpr int kTailLanes = 4;
+
+// one table entry (k - z)/s, correctly rounded, under the same conditions as build_table
+__device__ __forceinline__ float table_entry(float k, float s, float y, float z) {
+    if ((z == 0.0f || fabsf(z) >= 0x1p-60f) && s >= 0x1p-60f && s <= 0x1p30f) {
+        const float a = __fsub_rn(k, z);
+        const float q0 = __fmul_rn(a, y);
+        const float q1 = __fmaf_rn(__fmaf_rn(-q0, s, a), y, q0);
+        return __fmaf_rn(__fmaf_rn(-q1, s, a), y, q1);
+    }
+    return __fdiv_rn(__fsub_rn(k, z), s);
+}
+
+// the widest split of a group: every lane keeps at least one 8-element chunk and whole
+// 32-bit words of codes (1: no split)
+template <int NB, int P>
+struct TailMax {
+    static constexpr int a = NB * P / 32, b = P / 8;
+    static constexpr int value = (a < b ? a : b) > 16 ? 16 : (a < b ? a : b);
+};
+
+struct TailState {  // a segment's group, replicated in all of its lanes
+    int64_t cur;
+    SGroup gs;
+    int it;
+    bool act;
+};
+
+// One proximal round over a lane's E consecutive elements of its group (natural fp16 pairs),
+// with e = 0: returns the lane's pairwise partial sums and its code words.
+template <int NB, int E, bool CLIP>
+__device__ __forceinline__ void tail_round(const uint32_t (&h)[E / 2], float s, float z,
+                                           uint32_t tab_adj, float &esum, float &zsum,
+                                           uint32_t (&cw)[E * NB / 32]) {
+    constexpr int NCH = E / 8;
+    constexpr int LOGN = NCH == 1 ? 0 : NCH == 2 ? 1 : NCH == 4 ? 2 : NCH == 8 ? 3 : 4;
+    constexpr int CPW = 32 / NB;
+    constexpr float kQmax = (float)((1 << NB) - 1);
+    float sa[LOGN + 1], st[LOGN + 1];
+#pragma unroll
+    for (int ch = 0; ch < NCH; ++ch) {
+        float ar[8], tm[8];
+#pragma unroll
+        for (int m2 = 0; m2 < 8; m2 += 2) {
+            const float2 wp = __half22float2(*reinterpret_cast<const __half2 *>(&h[(8 * ch + m2) / 2]));
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int m = m2 + hh, j = 8 * ch + m;
+                const float w = hh ? wp.y : wp.x;
+                const float ws = __fmul_rn(w, s);
+                float t = __fadd_rn(ws, z);
+                if (CLIP) t = fminf(fmaxf(t, 0.0f), kQmax);
+                const float u = __fadd_rn(t, kMagic);
+                const float qf = __fsub_rn(u, kMagic);
+                const uint32_t bits = __float_as_uint(u);
+                const float what = lds_f32(tab_adj + (bits << 7));
+                uint32_t d;
+                asm("bfi.b32 %0, %1, %2, %3, %4;" : "=r"(d)
+                    : "r"(bits), "r"(j % CPW == 0 ? 0u : cw[j / CPW]), "r"(NB * (j % CPW)), "r"(NB));
+                cw[j / CPW] = d;
+                ar[m] = fabsf(__fsub_rn(w, what));
+                tm[m] = __fsub_rn(qf, ws);  // q - (W - 0) s
+            }
+        }
+        pw_push<LOGN>(sa, ch, tree8(ar));
+        pw_push<LOGN>(st, ch, tree8(tm));
+    }
+    esum = sa[LOGN];
+    zsum = st[LOGN];
+}
+
+// Runs the warp's groups in segments of L lanes until they are all done, or until few enough
+// remain for a split into segments of 2L lanes (owners then marks the lanes holding them).
+// owners on entry: the lanes whose ts holds a group; segment i takes the i-th of them.
+template <int NB, int P, int L>
+__device__ void tail_epoch(const QParams &Pm, TailState &ts, unsigned &owners, float *tabw,
+                           unsigned *acc_w, const float *thr_s, const double *beta_s,
+                           float thr_last) {
+    constexpr int E = P / L, CW = E * NB / 32, NQ = 1 << NB;
+    constexpr float kQmax = (float)(NQ - 1);
+    const int K = Pm.K;
+    const int lane = threadIdx.x & 31, seg = lane / L, l = lane % L;
+    const int n = __popc(owners);
+    const int pos = seg < n ? nth_set_bit(owners, seg) : -1;
+    const int src = pos >= 0 ? pos : lane;
+    TailState me;
+    me.cur = __shfl_sync(kFull, ts.cur, src);
+    me.gs.s = __shfl_sync(kFull, ts.gs.s, src);
+    me.gs.y = __shfl_sync(kFull, ts.gs.y, src);
+    me.gs.z = __shfl_sync(kFull, ts.gs.z, src);
+    me.gs.lo = __shfl_sync(kFull, ts.gs.lo, src);
+    me.gs.hi = __shfl_sync(kFull, ts.gs.hi, src);
+    me.gs.A = __shfl_sync(kFull, ts.gs.A, src);
+    me.it = __shfl_sync(kFull, ts.it, src);
+    me.act = pos >= 0;
+    uint32_t h[E / 2];
+    if (me.act) {  // this lane's slice of the row (in L2: the row was read a moment ago)
+        const uint4 *src_row = reinterpret_cast<const uint4 *>(Pm.W + me.cur * P + l * E);
+#pragma unroll
+        for (int v = 0; v < E / 8; ++v) {
+            const uint4 x = src_row[v];
+            h[4 * v] = x.x; h[4 * v + 1] = x.y; h[4 * v + 2] = x.z; h[4 * v + 3] = x.w;
+        }
+    } else {  // a segment without a group: zero row, zero state (inside every range)
+#pragma unroll
+        for (int i = 0; i < E / 2; ++i) h[i] = 0;
+        me.gs.idle();
+        me.it = 0;
+    }
+    // every lane looks up in its own column; lane l of a segment computes entries k = l, l + L,
+    // ... and writes each into all L columns of the segment (rotated, so the lanes of a
+    // segment store to L different banks at a time)
+    const uint32_t col = (uint32_t)__cvta_generic_to_shared(tabw + lane);
+    const uint32_t col0 = col - 4u * l;
+    const uint32_t tab_adj = col - (0x4B400000u << 7);
+    uint32_t cw[CW];
+#pragma unroll
+    for (int i = 0; i < CW; ++i) cw[i] = 0;
+    while (true) {
+        const int ri = min(me.it, K - 1);
+        __syncwarp();
+#pragma unroll
+        for (int kk = 0; kk < (NQ + L - 1) / L; ++kk) {
+            const int k = l + kk * L;
+            if (k < NQ) {
+                const float v = table_entry((float)k, me.gs.s, me.gs.y, me.gs.z);
+#pragma unroll
+                for (int i = 0; i < L; ++i) sts_f32(col0 + 4u * ((l + i) & (L - 1)) + 128u * k, v);
+            }
+        }
+        __syncwarp();
+        const float lz = __fadd_rn(me.gs.lo, me.gs.z), hz = __fadd_rn(me.gs.hi, me.gs.z);
+        const bool inside = lz >= -0.5f && hz < kQmax + 0.5f;
+        float esum, zsum;
+        if (__all_sync(kFull, inside))
+            tail_round<NB, E, false>(h, me.gs.s, me.gs.z, tab_adj, esum, zsum, cw);
+        else
+            tail_round<NB, E, true>(h, me.gs.s, me.gs.z, tab_adj, esum, zsum, cw);
+#pragma unroll
+        for (int off = 1; off < L; off <<= 1) {
+            esum = __fadd_rn(esum, __shfl_xor_sync(kFull, esum, off));
+            zsum = __fadd_rn(zsum, __shfl_xor_sync(kFull, zsum, off));
+        }
+        const float B = resid_bound(lz, hz, me.gs.A, me.gs.z, me.gs.y, kQmax);
+        const bool slow = me.act && B > thr_s[ri];
+        if (slow) zsum = group_zsum_shrink<NB>(Pm.W + me.cur * P, P, P, me.gs.s, me.gs.z, tab_adj, beta_s[ri], Pm.p);
+        const float znew = __fmul_rn(zsum, 1.0f / (float)P);
+        if (me.act) {
+            const bool done = (!slow && !(B > thr_last) && znew == me.gs.z) || me.it == K - 1;
+            if (l == 0) {
+                const u64 fx = err_fixed(esum);
+                add_fixed(acc_w + 4 * me.it, fx);
+                if (done && me.it + 1 < K) add_fixed(acc_w + 4 * (K + me.it + 1), fx);
+            }
+            if (done) {
+                uint32_t *dst = reinterpret_cast<uint32_t *>(Pm.packed) + me.cur * (P * NB / 32) + l * CW;
+#pragma unroll
+                for (int i = 0; i < CW; ++i) dst[i] = cw[i];
+                if (l == 0) stream_meta(Pm, me.cur, me.gs.s, me.gs.y, me.gs.z, me.it);
+                me.act = false;  // keeps its consistent row and state
+            } else {
+                me.gs.z = znew;
+                ++me.it;
+            }
+        }
+        const unsigned lead = __ballot_sync(kFull, l == 0 && me.act);
+        if (lead == 0 || (2 * L <= TailMax<NB, P>::value && __popc(lead) * 2 * L <= 32)) {
+            owners = lead;
+            ts = me;
+            return;
+        }
+    }
+}
+
+// the rest of the warp's groups: owners marks the lanes whose (cur, gs, it) hold one
+template <int NB, int P>
+__device__ __noinline__ void tail_run(const QParams &Pm, unsigned owners, int64_t cur, const SGroup &gs,
+                         int it, float *tabw, unsigned *acc_w, const float *thr_s,
+                         const double *beta_s, float thr_last) {
+    constexpr int LM = TailMax<NB, P>::value;
+    static_assert(LM >= 2, "no tail split for this group shape");
+    TailState ts;
+    ts.cur = cur;
+    ts.gs = gs;
+    ts.it = it;
+    ts.act = true;
+    while (owners) {
+        const int n = __popc(owners);
+        int L = 32;
+        while (L > 1 && n * L > 32) L >>= 1;
+        if (L > LM) L = LM;
+        if (L >= 16 && LM >= 16) tail_epoch<NB, P, (LM >= 16 ? 16 : 2)>(Pm, ts, owners, tabw, acc_w, thr_s, beta_s, thr_last);
+        else if (L >= 8 && LM >= 8) tail_epoch<NB, P, (LM >= 8 ? 8 : 2)>(Pm, ts, owners, tabw, acc_w, thr_s, beta_s, thr_last);
+        else if (L >= 4 && LM >= 4) tail_epoch<NB, P, (LM >= 4 ? 4 : 2)>(Pm, ts, owners, tabw, acc_w, thr_s, beta_s, thr_last);
+        else tail_epoch<NB, P, 2>(Pm, ts, owners, tabw, acc_w, thr_s, beta_s, thr_last);
+    }
+}
+
 template <int NB, int P>
 __global__ void __launch_bounds__(kThreads, P <= 64 ? 2 : 1) hqq_stream_kernel(const __grid_constant__ QParams Pm) {
     extern __shared__ __align__(16) unsigned char smem[];
@@ -1225,6 +1436,16 @@ __global__ void __launch_bounds__(kThreads, P <= 64 ? 2 : 1) hqq_stream_kernel(c
         }
         const bool active = cur >= 0;
         if (!__any_sync(kFull, active)) break;
+        if constexpr (TailMax<NB, P>::value >= 2) {
+            // nothing left to claim and at most kTailLanes groups left in the warp: split them
+            if (K > 0 && __all_sync(kFull, nxt < 0)) {
+                const unsigned owners = __ballot_sync(kFull, active);
+                if (__popc(owners) <= kTailLanes) {
+                    tail_run<NB, P>(Pm, owners, cur, gs, it, tabw, acc_w, thr_s, beta_s, thr_last);
+                    break;
+                }
+            }
+        }
         bool done = active && K == 0;
         if (__any_sync(kFull, active && K > 0)) {
             const int ri = min(it, max(K - 1, 0));

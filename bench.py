@@ -155,6 +155,21 @@ class ClockSampler:
                 "window": window, "power_w_max": max((num(p[3]) or 0.0) for p in win)}
 
 
+def shard(items, rank: int, ws: int):
+    """This rank's share of independent work items (every item on exactly one rank)."""
+    return items[rank::ws]
+
+
+def max_over_ranks(values, device, ws: int):
+    """Element-wise maximum of per-rank timings (a no-op on one rank)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if ws > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 def dist_setup():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -237,7 +252,7 @@ def run_stack(args, ws, rank, local):
         dist.init_process_group("nccl", device_id=dev,
                                 timeout=__import__("datetime").timedelta(seconds=120))
     keys = [(l, i) for l in range(wl.STACK_LAYERS) for i in range(len(wl.STACK_SHAPES))]
-    mine = keys[rank::ws]
+    mine = shard(keys, rank, ws)
     Ws = [wl.stack_matrix_torch(l, i, dev) for l, i in mine]
     outs = [hqq.hqq_quantize(W, NBITS, GROUP, AXIS, iters=ITERS, debug=True) for W in Ws]
     torch.cuda.synchronize()
@@ -280,10 +295,7 @@ def run_stack(args, ws, rank, local):
     ms = a.elapsed_time(b) / args.steps
     sampler.stop()
     clocks = sampler.summary(tw0, tw1)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if ws > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = t.item()
+    ms, = max_over_ranks([ms], dev, ws)
     n_all = sum(r * c for r, c in (wl.STACK_SHAPES[i] for _, i in keys))
     n_mine = sum(W.numel() for W in Ws)
     if rank == 0:
@@ -454,10 +466,7 @@ def main():
     clocks = sampler.summary(tw0, tw1)
 
     # max over ranks
-    t = torch.tensor([total_ms, q_ms, d_ms, e2e_ms, d_b2b_ms], dtype=torch.float64, device=dev)
-    if ws > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, q_ms, d_ms, e2e_ms, d_b2b_ms = t.tolist()
+    total_ms, q_ms, d_ms, e2e_ms, d_b2b_ms = max_over_ranks([total_ms, q_ms, d_ms, e2e_ms, d_b2b_ms], dev, ws)
 
     if rank == 0:
         pk = peaks()

@@ -1631,6 +1631,11 @@ __global__ void __launch_bounds__(kDqThreads) hqq_dequant_kernel(
     wait_prerequisite();  // the codes may come from the kernel launched just before
     allow_dependents();
     uint32_t wd[kDqU];
+    // MODE 3 (axis 1, g >= codes per word): a word spans at most two groups; both metadata
+    // pairs are loaded here, alongside the word, and codes c < cb belong to the first
+    float z0[MODE == 3 ? kDqU : 1], d0[MODE == 3 ? kDqU : 1], z1[MODE == 3 ? kDqU : 1],
+        d1[MODE == 3 ? kDqU : 1];
+    int cb[MODE == 3 ? kDqU : 1];
 #pragma unroll
     for (int u = 0; u < kDqU; ++u) {
         const int64_t wi = wbase + u * kDqThreads;
@@ -1643,6 +1648,16 @@ __global__ void __launch_bounds__(kDqThreads) hqq_dequant_kernel(
                 for (int b = 0; b < 4 && wi * 4 + b < packed_bytes; ++b)
                     wd[u] |= (uint32_t)pb[wi * 4 + b] << (8 * b);
             }
+            if constexpr (MODE == 3) {
+                const int64_t n0 = wi * CPW;
+                const int64_t k0 = wpg_shift >= 0 ? (n0 >> wpg_shift) : n0 / g;
+                const int64_t k1 = k0 + 1 < G ? k0 + 1 : k0;
+                cb[u] = (int)(g - (n0 - k0 * g));
+                z0[u] = __half2float(__ldg(zero + k0));
+                d0[u] = __half2float(__ldg(scale + k0));
+                z1[u] = __half2float(__ldg(zero + k1));
+                d1[u] = __half2float(__ldg(scale + k1));
+            }
         }
     }
 #pragma unroll
@@ -1652,7 +1667,14 @@ __global__ void __launch_bounds__(kDqThreads) hqq_dequant_kernel(
         const int64_t n0 = wi * CPW;
         uint32_t res[(CPW + 1) / 2];
         float v[CPW];
-        if (MODE == 0) {
+        if constexpr (MODE == 3) {
+#pragma unroll
+            for (int c = 0; c < CPW; ++c) {
+                const bool first = c < cb[u];
+                const float qf = __fsub_rn(__int_as_float(0x4B000000 | (int)((wd[u] >> (NB * c)) & MASK)), 8388608.0f);
+                v[c] = __fmul_rn(__fsub_rn(qf, first ? z0[u] : z1[u]), first ? d0[u] : d1[u]);
+            }
+        } else if (MODE == 0) {
             const int64_t k = wpg_shift >= 0 ? (wi >> wpg_shift) : (n0 / g);
             const float zf = __half2float(zero[k]), df = __half2float(scale[k]);
 #pragma unroll
@@ -1764,6 +1786,11 @@ cudaError_t launch_dequant(const uint8_t *pk, const __half *sc, const __half *ze
     // programmatic launch: overlaps the kernel before it, which the kernel waits for
     if (axis == 1 && g % CPW == 0)
         return launch_pdl(hqq_dequant_kernel<NB, 0>, blocks, kDqThreads, 0, st, pw, sc, ze, N, g, G, pb, shift, false, out);
+    if (axis == 1 && g >= CPW) {  // a word spans at most two groups
+        int gs = -1;
+        if ((g & (g - 1)) == 0) { gs = 0; while ((1 << gs) < g) ++gs; }
+        return launch_pdl(hqq_dequant_kernel<NB, 3>, blocks, kDqThreads, 0, st, pw, sc, ze, N, g, G, pb, gs, false, out);
+    }
     if (axis == 1)
         return launch_pdl(hqq_dequant_kernel<NB, 1>, blocks, kDqThreads, 0, st, pw, sc, ze, N, g, G, pb, -1, false, out);
     return launch_pdl(hqq_dequant_kernel<NB, 2>, blocks, kDqThreads, 0, st, pw, sc, ze, N, g, G, pb, -1, vec_meta, out);

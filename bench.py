@@ -421,17 +421,62 @@ def main():
     q_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
     d_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
 
-    # dequantize alone, back to back over the rotating buffers: its sustained throughput, without
-    # the per-call event brackets of the step loop (each adds about as much as a short launch)
+    # Dequantize alone and the fused forward product y = W_hat @ x, each timed back to back over
+    # the rotating buffers, plus the unfused path the fused one replaces: dequantize, then the
+    # library's fp16 x @ W_hat.T.  The loops are captured in a CUDA graph and replayed, so the
+    # host's per-call launch cost (Python + ctypes) is not what gets measured; without graph
+    # support the plain loop is timed instead.
+    import torch.nn.functional as F
     nb2b = max(2 * ROTATE, min(args.steps, 400))
-    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    b0.record(stream)
-    for i in range(nb2b):
-        hqq.hqq_dequantize(outs[i % ROTATE], out=deqs[i % ROTATE])
-    b1.record(stream)
-    torch.cuda.synchronize()
-    d_b2b_ms = b0.elapsed_time(b1) / nb2b
+    xv = torch.randn(COLS, device=dev).to(torch.float16)
+    yv = [torch.empty(ROWS, dtype=torch.float32, device=dev) for _ in range(ROTATE)]
+    yl = [torch.empty(1, ROWS, dtype=torch.float16, device=dev) for _ in range(ROTATE)]
+
+    def loop_dequant(n):
+        for i in range(n):
+            hqq.hqq_dequantize(outs[i % ROTATE], out=deqs[i % ROTATE])
+
+    def loop_gemv(n):
+        for i in range(n):
+            hqq.hqq_gemv(outs[i % ROTATE], xv, out=yv[i % ROTATE])
+
+    def loop_unfused(n):
+        for i in range(n):
+            k = i % ROTATE
+            hqq.hqq_dequantize(outs[k], out=deqs[k])
+            torch.matmul(xv.unsqueeze(0), deqs[k].t(), out=yl[k])
+
+    def per_call_ms(loop):
+        loop(2 * ROTATE)  # warm-up (library modules, cuBLAS handles)
+        torch.cuda.synchronize()
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        try:
+            side = torch.cuda.Stream(dev)
+            side.wait_stream(torch.cuda.current_stream(dev))
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(side):
+                with torch.cuda.graph(graph, stream=side):
+                    loop(nb2b)
+            torch.cuda.current_stream(dev).wait_stream(side)
+            graph.replay()
+            torch.cuda.synchronize()
+            b0.record(stream)
+            for _ in range(4):
+                graph.replay()
+            b1.record(stream)
+            torch.cuda.synchronize()
+            return b0.elapsed_time(b1) / (4 * nb2b), "cuda graph replay"
+        except RuntimeError:
+            torch.cuda.synchronize()
+            b0.record(stream)
+            loop(nb2b)
+            b1.record(stream)
+            torch.cuda.synchronize()
+            return b0.elapsed_time(b1) / nb2b, "plain loop"
+
+    d_b2b_ms, b2b_how = per_call_ms(loop_dequant)
+    gemv_ms, _ = per_call_ms(loop_gemv)
+    unfused_ms, _ = per_call_ms(loop_unfused)
 
     # end to end through the public API: pinned host W in, packed codes + metadata + dequantized
     # W out, copies inside the timed region
@@ -466,7 +511,8 @@ def main():
     clocks = sampler.summary(tw0, tw1)
 
     # max over ranks
-    total_ms, q_ms, d_ms, e2e_ms, d_b2b_ms = max_over_ranks([total_ms, q_ms, d_ms, e2e_ms, d_b2b_ms], dev, ws)
+    total_ms, q_ms, d_ms, e2e_ms, d_b2b_ms, gemv_ms, unfused_ms = max_over_ranks(
+        [total_ms, q_ms, d_ms, e2e_ms, d_b2b_ms, gemv_ms, unfused_ms], dev, ws)
 
     if rank == 0:
         pk = peaks()
@@ -507,7 +553,13 @@ def main():
             "dequant_gbs": hbm_d, "dequant_hbm_frac": hbm_d / pk["hbm_gbs"],
             "dequant_back_to_back": {"us": d_b2b_ms * 1e3, "gbs": alg_bytes / (d_b2b_ms / 1e3) / 1e9,
                                      "hbm_frac": alg_bytes / (d_b2b_ms / 1e3) / 1e9 / pk["hbm_gbs"],
-                                     "launches": nb2b},
+                                     "launches": nb2b, "timed_by": b2b_how},
+            "gemv": {"us": gemv_ms * 1e3,
+                     "gbs": (packed_bytes + 4 * G + 2 * COLS + 4 * ROWS) / (gemv_ms / 1e3) / 1e9,
+                     "hbm_frac": (packed_bytes + 4 * G + 2 * COLS + 4 * ROWS) / (gemv_ms / 1e3) / 1e9 / pk["hbm_gbs"],
+                     "alg_bytes_per_launch": packed_bytes + 4 * G + 2 * COLS + 4 * ROWS,
+                     "unfused_dequant_then_matmul_us": unfused_ms * 1e3, "launches": nb2b,
+                     "timed_by": b2b_how},
             "hbm_peak_gbs": pk["hbm_gbs"], "hbm_peak_src": pk["src"],
             "alg_bytes_per_launch": alg_bytes,
             "roofline": roofline,

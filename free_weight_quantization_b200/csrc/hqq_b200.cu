@@ -1796,6 +1796,161 @@ cudaError_t launch_dequant(const uint8_t *pk, const __half *sc, const __half *ze
     return launch_pdl(hqq_dequant_kernel<NB, 2>, blocks, kDqThreads, 0, st, pw, sc, ze, N, g, G, pb, -1, vec_meta, out);
 }
 
+
+// ==========================================================================================
+// The quantized layer's forward product for one input vector [HQQ 算法解读,
+// "从压缩文件到一次前向"]: unpack -> (q - zero) * scale -> x @ W_hat.T, fused so that W_hat never
+// reaches memory.  Each W_hat[r, c] is the exact fp16 value hqq_dequantize writes; the product
+// with the fp16 x[c] is exact in binary32, and the row sum runs in binary32.
+// ==========================================================================================
+
+// Axis 1, 2- or 4-bit, cols and g multiples of the codes per word: one warp per output row.
+// Lane l takes the row's words l, l + 32, ... (every warp load covers 128 contiguous bytes) and
+// loads kGvU of them, with their metadata, before using any: a 4096-column 4-bit row is one
+// batch, so a warp waits for memory once.  A word's codes are dequantized in pairs exactly as
+// hqq_dequantize does (a code c becomes 2^23 + c by a byte permute against 0x4B000000, then
+// (q - z) * Delta in binary32, rounded to fp16) and multiplied with x in packed binary32 FMAs.
+constexpr int kGvU = 16;
+
+template <int NB>
+__device__ __forceinline__ float2 gemv_word(uint32_t w, float zf, float df, const __half *xw,
+                                            float2 acc) {
+    const float2 nm = make_float2(-8388608.0f, -8388608.0f), nz = make_float2(-zf, -zf);
+    const float2 d2 = make_float2(df, df);
+    constexpr int CPW = Pack<NB>::cpw;
+    uint32_t xs[CPW / 2];
+#pragma unroll
+    for (int v = 0; v < CPW / 8; ++v) {
+        const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(xw) + v);
+        xs[4 * v] = xv.x; xs[4 * v + 1] = xv.y; xs[4 * v + 2] = xv.z; xs[4 * v + 3] = xv.w;
+    }
+    if constexpr (NB == 4) {
+        const uint32_t ev = w & 0x0F0F0F0Fu, od = (w >> 4) & 0x0F0F0F0Fu;  // codes 2i, 2i+1 in byte i
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 q = make_float2(__uint_as_float(__byte_perm(ev, 0x4B000000u, 0x7540u + i)),
+                                         __uint_as_float(__byte_perm(od, 0x4B000000u, 0x7540u + i)));
+            const float2 v = __fmul2_rn(__fadd2_rn(__fadd2_rn(q, nm), nz), d2);
+            const float2 xf = __half22float2(*reinterpret_cast<const __half2 *>(&xs[i]));
+            acc = __ffma2_rn(__half22float2(__floats2half2_rn(v.x, v.y)), xf, acc);
+        }
+    } else {  // 2 bit: field s of byte b is code 4b + s
+        uint32_t f[4];
+#pragma unroll
+        for (int s = 0; s < 4; ++s) f[s] = (w >> (2 * s)) & 0x03030303u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {  // codes 2i, 2i+1: byte i/2, fields 2(i%2) and +1
+            const int b = i >> 1, s = 2 * (i & 1);
+            const float2 q = make_float2(__uint_as_float(__byte_perm(f[s], 0x4B000000u, 0x7540u + b)),
+                                         __uint_as_float(__byte_perm(f[s + 1], 0x4B000000u, 0x7540u + b)));
+            const float2 v = __fmul2_rn(__fadd2_rn(__fadd2_rn(q, nm), nz), d2);
+            const float2 xf = __half22float2(*reinterpret_cast<const __half2 *>(&xs[i]));
+            acc = __ffma2_rn(__half22float2(__floats2half2_rn(v.x, v.y)), xf, acc);
+        }
+    }
+    return acc;
+}
+
+template <int NB>
+__global__ void __launch_bounds__(256) hqq_gemv_kernel(const uint32_t *__restrict__ packed,
+                                                       const __half *__restrict__ scale,
+                                                       const __half *__restrict__ zero,
+                                                       int64_t rows, int wpr, int gpr,
+                                                       int wpg_shift, int wpg,
+                                                       const __half *__restrict__ x,
+                                                       float *__restrict__ y) {
+    constexpr int CPW = Pack<NB>::cpw;
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    wait_prerequisite();  // codes and x may come from the kernel launched just before
+    allow_dependents();
+    if (row >= rows) return;  // whole warps
+    const uint32_t *prow = packed + row * wpr;
+    const int64_t k0 = row * gpr;
+    float2 acc = make_float2(0.0f, 0.0f);
+    for (int w0 = lane; w0 < wpr; w0 += 32 * kGvU) {
+        uint32_t wd[kGvU];
+        float zf[kGvU], df[kGvU];
+#pragma unroll
+        for (int u = 0; u < kGvU; ++u) {
+            const int w = w0 + 32 * u;
+            wd[u] = 0;
+            zf[u] = 0.0f;
+            df[u] = 0.0f;
+            if (w < wpr) {
+                const int64_t k = k0 + (wpg_shift >= 0 ? (w >> wpg_shift) : w / wpg);
+                wd[u] = __ldcs(prow + w);
+                zf[u] = __half2float(__ldg(zero + k));
+                df[u] = __half2float(__ldg(scale + k));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kGvU; ++u) {
+            const int w = w0 + 32 * u;
+            if (w < wpr) acc = gemv_word<NB>(wd[u], zf[u], df[u], x + (int64_t)w * CPW, acc);
+        }
+    }
+    float s = __fadd_rn(acc.x, acc.y);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s = __fadd_rn(s, __shfl_xor_sync(kFull, s, off));
+    if (lane == 0) y[row] = s;
+}
+
+// Any other layout: one warp per output row, each lane takes columns lane, lane + 32, ...
+// and reads its codes one at a time (flat row-major code order, groups by axis).
+template <int NB>
+__global__ void __launch_bounds__(256) hqq_gemv_any_kernel(const uint8_t *__restrict__ packed,
+                                                           const __half *__restrict__ scale,
+                                                           const __half *__restrict__ zero,
+                                                           int64_t rows, int64_t cols, int64_t g,
+                                                           int64_t G, int axis,
+                                                           const __half *__restrict__ x,
+                                                           float *__restrict__ y) {
+    constexpr uint32_t MASK = (1u << NB) - 1u;
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    wait_prerequisite();
+    allow_dependents();
+    if (row >= rows) return;
+    float acc = 0.0f;
+    for (int64_t c = lane; c < cols; c += 32) {
+        const int64_t n = row * cols + c;
+        uint32_t q;
+        if (NB == 3) {
+            const uint32_t wv = __ldg(reinterpret_cast<const uint32_t *>(packed) + n / 10);
+            q = (wv >> (3 * (int)(n % 10))) & MASK;
+        } else {
+            const int per = 8 / NB;
+            q = ((uint32_t)__ldg(packed + n / per) >> (NB * (int)(n % per))) & MASK;
+        }
+        const int64_t k = axis == 1 ? n / g : n % G;
+        const float v = __fmul_rn(__fsub_rn((float)q, __half2float(__ldg(zero + k))), __half2float(__ldg(scale + k)));
+        acc = __fmaf_rn(__half2float(__float2half_rn(v)), __half2float(__ldg(x + c)), acc);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(kFull, acc, off));
+    if (lane == 0) y[row] = acc;
+}
+
+template <int NB>
+cudaError_t launch_gemv(const uint8_t *pk, const __half *sc, const __half *ze, int64_t rows,
+                        int64_t cols, int64_t g, int64_t G, int axis, const __half *x, float *y,
+                        cudaStream_t st) {
+    constexpr int CPW = Pack<NB>::cpw;
+    const unsigned blocks = (unsigned)((rows + 7) / 8);
+    const int64_t wpr = cols / CPW;
+    if (NB != 3 && axis == 1 && cols % CPW == 0 && g % CPW == 0 && ((uintptr_t)x & 15) == 0 &&
+        wpr < ((int64_t)1 << 30)) {
+        const int wpg = (int)(g / CPW);
+        int shift = -1;
+        if ((wpg & (wpg - 1)) == 0) { shift = 0; while ((1 << shift) < wpg) ++shift; }
+        return launch_pdl(hqq_gemv_kernel<NB>, blocks, 256, 0, st, (const uint32_t *)pk, sc, ze,
+                          rows, (int)wpr, (int)(cols / g), shift, wpg, x, y);
+    }
+    return launch_pdl(hqq_gemv_any_kernel<NB>, blocks, 256, 0, st, pk, sc, ze, rows, cols, g, G,
+                      axis, x, y);
+}
+
 // ------------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------------
@@ -2090,6 +2245,28 @@ extern "C" int hqq_dequantize(const void *packed, const void *scale, const void 
     case 4: e = launch_dequant<4>(pk, sc, ze, pl.N, pl.g, pl.G, axis, pb, out, st); break;
     case 3: e = launch_dequant<3>(pk, sc, ze, pl.N, pl.g, pl.G, axis, pb, out, st); break;
     default: e = launch_dequant<2>(pk, sc, ze, pl.N, pl.g, pl.G, axis, pb, out, st); break;
+    }
+    return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
+}
+
+extern "C" int hqq_gemv(const void *packed, const void *scale, const void *zero, int64_t rows,
+                        int64_t cols, int nbits, int64_t group_size, int axis, const void *x,
+                        float *y, void *stream) {
+    Plan pl;
+    int rc = make_plan(rows, cols, nbits, group_size, axis, 0, &pl);
+    if (rc != HQQ_OK) return rc;
+    if (!packed || !scale || !zero || !x || !y) return HQQ_ERR_ARG;
+    if (!aligned_to(packed, 16) || !aligned_to(scale, 2) || !aligned_to(zero, 2) ||
+        !aligned_to(x, 2) || !aligned_to(y, 4))
+        return HQQ_ERR_ALIGN;
+    cudaStream_t st = (cudaStream_t)stream;
+    const uint8_t *pk = (const uint8_t *)packed;
+    const __half *sc = (const __half *)scale, *ze = (const __half *)zero, *xh = (const __half *)x;
+    cudaError_t e;
+    switch (nbits) {
+    case 4: e = launch_gemv<4>(pk, sc, ze, rows, cols, pl.g, pl.G, axis, xh, y, st); break;
+    case 3: e = launch_gemv<3>(pk, sc, ze, rows, cols, pl.g, pl.G, axis, xh, y, st); break;
+    default: e = launch_gemv<2>(pk, sc, ze, rows, cols, pl.g, pl.G, axis, xh, y, st); break;
     }
     return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
 }

@@ -44,6 +44,7 @@ SIGNATURES = {
     "hqq_dequantize": (_I32, [_P, _P, _P, _I64, _I64, _I32, _I64, _I32, _P, _P]),
     "hqq_quantize_noalloc": (_I32, [_P, _I64, _I64, _I32, _I64, _I32, ctypes.POINTER(HqqOpt), _P,
                                     _P, _P, _P, _P, _P, _P, _P, _P]),
+    "hqq_gemv": (_I32, [_P, _P, _P, _I64, _I64, _I32, _I64, _I32, _P, _P, _P]),
     "hqq_strerror": (ctypes.c_char_p, [_I32]),
 }
 
@@ -188,6 +189,21 @@ def hqq_dequantize(q: Quantized, out: torch.Tensor | None = None,
     rc = lib().hqq_dequantize(_ptr(q.packed), _ptr(q.scale), _ptr(q.zero), q.rows, q.cols, q.nbits,
                               q.group_size, q.axis, _ptr(out), ctypes.c_void_p(st.cuda_stream))
     _check(rc, "hqq_dequantize")
+    return out
+
+
+def hqq_gemv(q: Quantized, x: torch.Tensor, out: torch.Tensor | None = None,
+             stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """y = W_hat @ x with dequantization fused in (see hqq_gemv in the header): x is a
+    contiguous fp16 CUDA vector of q.cols entries, y a binary32 vector of q.rows."""
+    if x.dtype != torch.float16 or not x.is_cuda or x.dim() != 1 or x.numel() != q.cols or not x.is_contiguous():
+        raise HqqError("x must be a contiguous fp16 CUDA vector with cols entries")
+    if out is None:
+        out = torch.empty(q.rows, dtype=torch.float32, device=q.packed.device)
+    st = stream if stream is not None else torch.cuda.current_stream(q.packed.device)
+    rc = lib().hqq_gemv(_ptr(q.packed), _ptr(q.scale), _ptr(q.zero), q.rows, q.cols, q.nbits,
+                        q.group_size, q.axis, _ptr(x), _ptr(out), ctypes.c_void_p(st.cuda_stream))
+    _check(rc, "hqq_gemv")
     return out
 
 

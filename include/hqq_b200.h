@@ -126,6 +126,27 @@ int hqq_dequantize(const void *packed, const void *scale, const void *zero, int6
                    void *stream);
 
 /*
+ * hqq_gemv: the quantized layer's forward product for one input vector, with dequantization
+ * fused in [HQQ 算法解读, "从压缩文件到一次前向"]: unpack -> (q - zero) * scale -> x @ W_hat.T,
+ * without writing W_hat to memory.
+ *     y[r] = sum_c W_hat[r, c] * x[c]
+ * W_hat[r, c] is exactly the fp16 value hqq_dequantize writes. Each product of two fp16 values
+ * is exact in binary32, and the row sum runs in binary32 in an order of the kernel's choosing,
+ * so y[r] is within cols * 2^-23 * sum_c |W_hat[r, c] * x[c]| of the exact sum.
+ *   packed, scale, zero  as written by hqq_quantize for the same rows, cols, nbits, group_size
+ *                        and axis (packed 16-byte aligned, scale and zero 2-byte aligned)
+ *   x       [cols] fp16, 2-byte aligned. 16-byte alignment enables the fast path.
+ *   y       [rows] binary32, 4-byte aligned (output)
+ *   stream  cudaStream_t, or NULL for the default stream
+ * Every layout is accepted. The fast path (one warp per output row) needs axis 1, 2- or 4-bit
+ * codes, and cols and group_size multiples of the codes per 32-bit word (8 at 4 bit, 16 at 2
+ * bit). Other layouts read their codes one at a time.
+ * Returns HQQ_OK, HQQ_ERR_ARG (shape or null pointer), HQQ_ERR_ALIGN, or HQQ_ERR_CUDA.
+ */
+int hqq_gemv(const void *packed, const void *scale, const void *zero, int64_t rows, int64_t cols,
+             int nbits, int64_t group_size, int axis, const void *x, float *y, void *stream);
+
+/*
  * hqq_quantize without a workspace argument.  The pages have no counterpart to this call: it
  * exists for callers that cannot allocate device memory, such as plugins running inside a
  * framework whose pool owns all of the GPU's memory, or loops that must never call cudaMalloc

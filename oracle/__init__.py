@@ -69,6 +69,7 @@ def _load():
     lib.hqo_unpack.argtypes = [P, i64, i32, P]
     lib.hqo_unpack.restype = None
     lib.hqo_dequant.argtypes = [P, P, P, i64, i64, i32, i64, i32, P]
+    lib.hqo_gemv.argtypes = [P, P, P, i64, i64, i32, i64, i32, P, P, P]
     lib.hqo_dequant.restype = i32
     _lib = lib
     return lib
@@ -182,6 +183,24 @@ def quantize(W, nbits: int, group_size: int, axis: int = 1, iters: int = 20, lp_
                 packed=pack(codes, nbits), iters_run=n_run, err_trace=err,
                 mae_trace=[float(x) for x in mae[:n_run]], rows=rows, cols=cols, nbits=nbits,
                 group_size=group_size, axis=axis)
+
+
+def gemv(packed, scale, zero, rows: int, cols: int, nbits: int, group_size: int, axis: int,
+         x) -> tuple[np.ndarray, np.ndarray]:
+    """y = W_hat @ x in binary64 (W_hat the fp16 dequantized weights, x fp16 [cols]) and the
+    per-row sum of |W_hat * x|; see hqo_gemv."""
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    sc = _as_u16(scale)
+    ze = _as_u16(zero)
+    xh = _as_u16(x)
+    assert xh.size == cols
+    y = np.zeros(rows, np.float64)
+    mag = np.zeros(rows, np.float64)
+    rc = _load().hqo_gemv(_ptr(packed), _ptr(sc), _ptr(ze), rows, cols, nbits, group_size, axis,
+                          _ptr(xh), _ptr(y), _ptr(mag))
+    if rc != 0:
+        raise ValueError(f"oracle rejected the arguments (code {rc})")
+    return y, mag
 
 
 def dequant(packed, scale, zero, rows: int, cols: int, nbits: int, group_size: int,

@@ -23,6 +23,8 @@
  *                       quantize once more with the original W
  *   packing ........... [HQQ 算法解读, "为什么一定要分组"] two 4-bit codes per byte, four 2-bit
  *                       codes per byte, ten 3-bit codes per 32-bit word
+ *   forward product ... [HQQ 算法解读, "从压缩文件到一次前向"] unpack -> (q - zero)*scale ->
+ *                       x @ W_hat.T (hqo_gemv, one input vector)
  *
  * Readings taken where the page is silent (each is also listed in the design notes):
  *   - arithmetic is IEEE binary32, round-to-nearest-even, every product and sum rounded
@@ -355,5 +357,39 @@ int hqo_dequant(const uint8_t *packed, const uint16_t *scale_h, const uint16_t *
         W_out[n] = hqo_float_to_half(v);
     }
     free(codes);
+    return 0;
+}
+
+/*
+ * The quantized layer's forward product for one input vector [HQQ 算法解读,
+ * "从压缩文件到一次前向"]: unpack, (q - z)*Delta, then x @ W_hat.T, i.e.
+ *     y[r] = sum_c W_hat[r, c] * x[c]
+ * with W_hat exactly the fp16 values hqo_dequant produces and x fp16 [cols].  Every product of
+ * two fp16 values is exact in binary64, and the sum runs in binary64 in column order, so y
+ * carries only the rounding of that sum (the reading: the pages fix no summation order or
+ * precision for this step).  absum[r] = sum_c |W_hat[r, c] * x[c]| bounds any other
+ * summation order's error.  Both outputs [rows] binary64.
+ */
+int hqo_gemv(const uint8_t *packed, const uint16_t *scale_h, const uint16_t *zero_h,
+             int64_t rows, int64_t cols, int nbits, int64_t g, int axis, const uint16_t *x_h,
+             double *y, double *absum)
+{
+    if (hqo_check_args(rows, cols, nbits, g, axis)) return 1;
+    int64_t N = rows * cols;
+    uint16_t *w = (uint16_t *)malloc((size_t)N * sizeof(uint16_t));
+    if (!w) return 2;
+    int rc = hqo_dequant(packed, scale_h, zero_h, rows, cols, nbits, g, axis, w);
+    if (rc) { free(w); return rc; }
+    for (int64_t r = 0; r < rows; r++) {
+        double acc = 0.0, mag = 0.0;
+        for (int64_t c = 0; c < cols; c++) {
+            double p = (double)hqo_half_to_float(w[r * cols + c]) * (double)hqo_half_to_float(x_h[c]);
+            acc += p;
+            mag += fabs(p);
+        }
+        y[r] = acc;
+        absum[r] = mag;
+    }
+    free(w);
     return 0;
 }

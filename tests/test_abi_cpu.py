@@ -117,3 +117,23 @@ def test_strerror(L):
     for code in range(6):
         assert L.hqq_strerror(code)
     assert L.hqq_strerror(99) == b"unknown error"
+
+
+def test_gemv_rejects_on_host(L):
+    P = ctypes.c_void_p
+    gv = L.hqq_gemv
+    args = lambda **k: dict(dict(pk=FAKE, sc=FAKE, ze=FAKE, rows=64, cols=64, nb=4, g=64, ax=1,
+                                 x=FAKE, y=FAKE), **k)
+
+    def call(**k):
+        a = args(**k)
+        return gv(P(a["pk"]), P(a["sc"]), P(a["ze"]), a["rows"], a["cols"], a["nb"], a["g"],
+                  a["ax"], P(a["x"]) if a["x"] else None, P(a["y"]) if a["y"] else None, None)
+    assert call(nb=5) == 1
+    assert call(g=48) == 1                 # 4096 % 48 != 0
+    assert call(ax=2) == 1
+    assert call(x=0) == 1
+    assert call(y=0) == 1
+    assert call(pk=FAKE + 4) == 2          # packed not 16-byte aligned
+    assert call(x=FAKE + 1) == 2
+    assert call(y=FAKE + 2) == 2

@@ -361,3 +361,57 @@ def test_dequant_axis0_layout():
     r1 = oracle.quantize(Wt, 4, g, axis=1, iters=5)
     d1 = oracle.dequant(r1["packed"], r1["scale"], r1["zero"], Wt.shape[0], g, 4, g, axis=1)
     assert np.array_equal(d0.reshape(g, -1), d1.T)
+
+
+# ---- the forward product y = W_hat @ x [HQQ 算法解读, "从压缩文件到一次前向"] ----
+
+def _random_quantized(rows, cols, nbits, g, axis, seed):
+    r = np.random.default_rng(seed)
+    N = rows * cols
+    codes = r.integers(0, 1 << nbits, N).astype(np.uint8)
+    G = N // g
+    scale = (r.random(G) * 0.05 + 1e-3).astype(np.float16)
+    zero = (r.random(G) * (1 << nbits)).astype(np.float16)
+    return oracle.pack(codes, nbits), scale, zero
+
+
+@pytest.mark.parametrize("nbits,g,axis", [(4, 64, 1), (3, 64, 1), (2, 16, 1), (4, 32, 0)])
+def test_gemv_unit_vectors_give_the_dequantized_columns(nbits, g, axis):
+    # x = 2^-3 e_j picks column j of W_hat, scaled exactly: no rounding anywhere
+    rows, cols = 48, 128
+    packed, scale, zero = _random_quantized(rows, cols, nbits, g, axis, 5)
+    Wh = oracle.dequant(packed, scale, zero, rows, cols, nbits, g, axis).astype(np.float64)
+    for j in (0, 1, 77, cols - 1):
+        x = np.zeros(cols, np.float16)
+        x[j] = 0.125
+        y, mag = oracle.gemv(packed, scale, zero, rows, cols, nbits, g, axis, x)
+        assert np.array_equal(y, Wh[:, j] * 0.125)
+        assert np.array_equal(mag, np.abs(Wh[:, j]) * 0.125)
+
+
+def test_gemv_constant_codes_closed_form():
+    # every code k, one (Delta, z) for all groups: W_hat is the constant fp16((k - z) Delta), so
+    # y[r] = W_hat * sum(x); x on a 1/8 grid keeps every sum exact in binary64
+    rows, cols, nbits, g, k = 16, 256, 4, 64, 11
+    codes = np.full(rows * cols, k, np.uint8)
+    G = rows * cols // g
+    scale = np.full(G, 0.0123, np.float16)
+    zero = np.full(G, 7.25, np.float16)
+    packed = oracle.pack(codes, nbits)
+    x = (np.random.default_rng(3).integers(-32, 33, cols) / 8.0).astype(np.float16)
+    w0 = float(np.float16((np.float32(k) - np.float32(zero[0])) * np.float32(scale[0])))
+    y, _ = oracle.gemv(packed, scale, zero, rows, cols, nbits, g, 1, x)
+    assert np.array_equal(y, np.full(rows, w0 * float(x.astype(np.float64).sum())))
+
+
+def test_gemv_is_linear_in_x():
+    # with x on a coarse grid every partial sum is exact, so linearity holds bit for bit
+    rows, cols, nbits, g = 32, 192, 4, 64
+    packed, scale, zero = _random_quantized(rows, cols, nbits, g, 1, 9)
+    r = np.random.default_rng(4)
+    x1 = (r.integers(-8, 9, cols) / 4.0).astype(np.float16)
+    x2 = (r.integers(-8, 9, cols) / 4.0).astype(np.float16)
+    y1, _ = oracle.gemv(packed, scale, zero, rows, cols, nbits, g, 1, x1)
+    y2, _ = oracle.gemv(packed, scale, zero, rows, cols, nbits, g, 1, x2)
+    y12, _ = oracle.gemv(packed, scale, zero, rows, cols, nbits, g, 1, (x1 + x2).astype(np.float16))
+    assert np.array_equal(y12, y1 + y2)

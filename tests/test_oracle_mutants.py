@@ -40,6 +40,9 @@ MUTANTS = {
     "dequant adds z": ("float v = ((float)codes[n] - zf) * df;", "float v = ((float)codes[n] + zf) * df;"),
     "half truncates": ("float m = rintf(ldexpf(a, 10 - expo));", "float m = truncf(ldexpf(a, 10 - expo));"),
     "delta not inverted": ("scale_h[k] = hqo_float_to_half(1.0f / s[k]);", "scale_h[k] = hqo_float_to_half(s[k]);"),
+    "gemv transposed": ("(double)hqo_half_to_float(w[r * cols + c])", "(double)hqo_half_to_float(w[(c * rows + r) % N])"),
+    "gemv x reversed": ("(double)hqo_half_to_float(x_h[c]);", "(double)hqo_half_to_float(x_h[cols - 1 - c]);"),
+    "gemv signed magnitude": ("mag += fabs(p);", "mag += p;"),
 }
 
 

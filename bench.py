@@ -65,17 +65,28 @@ PROFILE = os.path.join(ROOT, "profiles", "hqq_stream_kernel_4096x4096_b4g64.md")
 KERNEL_SRC = os.path.join(ROOT, "free_weight_quantization_b200", "csrc", "hqq_b200.cu")
 
 
-def profiled_traffic():
-    """DRAM bytes per launch of the search kernel from the committed ncu summary, or None
-    when the kernel source has changed since that capture."""
+def code_hash(path: str) -> str:
+    """sha256 of a C/CUDA source with its comments and blank space removed, so that only a
+    change of code (not of a comment) makes a recorded profile stale."""
     import hashlib
+    import re
+    src = open(path, encoding="utf-8").read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    src = "\n".join(line.strip() for line in src.splitlines() if line.strip())
+    return hashlib.sha256(src.encode("utf-8")).hexdigest()
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the stream kernel from the committed ncu summary, or None
+    when the kernel source's code has changed since that capture."""
     try:
         text = open(PROFILE).read()
-        src = hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()
+        src = code_hash(KERNEL_SRC)
     except OSError:
         return None
-    fields = dict(l.split(":", 1) for l in text.splitlines() if l.startswith(("source-sha256:", "traffic-bytes-per-launch:")))
-    if fields.get("source-sha256", "").strip() != src:
+    fields = dict(l.split(":", 1) for l in text.splitlines() if l.startswith(("code-sha256:", "traffic-bytes-per-launch:")))
+    if fields.get("code-sha256", "").strip() != src:
         return None
     try:
         return float(fields["traffic-bytes-per-launch"])

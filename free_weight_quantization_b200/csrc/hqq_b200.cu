@@ -4,29 +4,35 @@
 // (ludovicoyin.github.io/blog/posts/hqq-half-quadratic-quantization), cited as
 // [HQQ 算法解读, <section>].  The arithmetic reproduces, operation for operation, the binary32
 // definition stated in include/hqq_b200.h: every product and sum rounded separately
-// (__fmul_rn/__fadd_rn, no contraction), IEEE division for W_hat = (q - z)/s, round half to
-// even, pairwise (recursive-halving) group sums, the lp shrink in binary64, and an exact
-// fixed-point (2^-32) 128-bit tensor-wide error sum for the stop rule.
+// (__fmul_rn/__fadd_rn and their packed .f32x2 forms, no contraction), W_hat = (q - z)/s
+// correctly rounded (a reciprocal product with Markstein's remainder corrections gives the
+// same bits as IEEE division), round half to even, pairwise (recursive-halving) group sums,
+// the lp shrink in binary64, and an exact fixed-point (2^-32) 128-bit tensor-wide error sum
+// for the stop rule.
 //
 // Design (no tensor cores: nothing here is a dense contraction; the loop is ALU-bound):
-//   search kernel  one CTA per tile of ~10k weights.  The tile is read from HBM once with
-//                  16-byte loads and kept in shared memory as binary32, one padded row per
-//                  group.  Warps are split into segments of L = P/16 lanes (P = group size
-//                  rounded up to a power of two >= 16); each lane holds 16 consecutive
-//                  elements of its group in registers, so a group's pairwise sums are a
-//                  16-element in-lane tree plus log2(L) xor-shuffle levels.  A segment runs
-//                  its group round after round until the zero stops moving (z_{i+1} == z_i
-//                  with every residual below the last round's shrink threshold: every later
-//                  round would repeat it exactly) or `iters` rounds are done, then takes the
-//                  next group of the tile from a shared counter, so finished groups free
-//                  their lanes.  Each round's per-group error goes to exact per-round
-//                  accumulators (a frozen group's error is carried to all later rounds with a
-//                  difference array).  The group's codes for its last round are packed with
-//                  the rest of the tile and written once.
-//   fixup kernel   evaluates the stop rule from the accumulators.  A group whose own last
-//                  round lies beyond the global stopping point is stale; only tiles holding a
-//                  stale group are recomputed (replaying exactly min(b, f) zero updates).
-//   dequant kernel one thread per 16 packed bytes, 16-byte loads and stores.
+//   A quantize call launches a one-block zero kernel for the round sums, then one of two
+//   engines and a fixup kernel, each later kernel with programmatic stream serialization so
+//   that its launch overlaps the kernel before it (griddepcontrol.wait orders the data).
+//   stream engine  axis 1, 2- or 4-bit codes, power-of-two groups of 16..128 that fill whole
+//                  32-bit words: a persistent kernel with one group per lane.  The lane
+//                  keeps the group's fp16 row in registers for all its rounds, its table of
+//                  the 2^b reconstructions in its own shared-memory column, and the next
+//                  group's row in a swizzled shared-memory slot (cp.async, one group ahead).
+//                  Groups come from a global counter; once it is empty, idle lanes take the
+//                  queued groups of busy ones, and a warp's last few groups are split over
+//                  segments of lanes.
+//   tile engine    everything else (axis 0, 3-bit, other group sizes): one CTA per tile of
+//                  groups staged in shared memory, segments of L = P/16 lanes per group.
+//   Both engines run a group round after round until its zero stops moving (z_{i+1} == z_i
+//   with every residual provably below the last round's shrink threshold: every later round
+//   would repeat it exactly) or `iters` rounds are done; a group's error goes to exact
+//   per-round counters (a frozen group's error is carried to later rounds by a difference
+//   array), and its last round's codes are its final codes.  The last CTA to finish applies
+//   the stop rule; the fixup kernel recomputes the few groups whose own last round lies past
+//   the kept one, replaying exactly min(b, f) zero updates.
+//   dequant        one packed 32-bit word per lane per step, coalesced loads and stores.
+//   gemv           dequantize fused into y = W_hat @ x for one input vector.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>

@@ -198,7 +198,10 @@ def run_reference(args, ws, rank):
     from free_weight_quantization_b200 import workloads as wl
     oracle.build()
     W = CASE.make()
-    rows = min(256, ROWS)             # each step: a slice of up to 256 rows of the matrix
+    # each step is a slice of up to 256 rows, fewer for long runs, so the whole run stays
+    # within about two minutes: the oracle needs about 2 ms per 4096 weights of a row
+    budget_rows = int(60000 * 4096 / COLS)
+    rows = max(1, min(256, ROWS, budget_rows // (args.warmup + args.steps)))
     times = []
     for i in range(args.warmup + args.steps):
         nsl = ROWS // rows

@@ -98,9 +98,10 @@ size_t hqq_quantize_workspace_bytes(int64_t rows, int64_t cols, int nbits, int64
  *                over groups of floor(2^32 * sum_group |W - W_hat|) at round i, as
  *                (low 64 bits, high 64 bits); MAE_i = that / 2^32 / N.  Entries at or past
  *                iters_run are unspecified.
- *   group_rounds [G] uint8, nullable (output): rounds each group needed before its zero
- *                stopped moving (a later round would repeat the last one exactly), at most
- *                iters; 0 when iters = 0.  Diagnostic: the work the loop really required.
+ *   group_rounds [G] uint8, nullable (output): rounds each group ran.  A group stops once
+ *                its zero stops moving and every later round provably repeats the last one,
+ *                or after iters rounds; 0 when iters = 0.  Diagnostic: the work the loop
+ *                did.
  *   workspace    >= hqq_quantize_workspace_bytes(...) bytes, 16-byte aligned; contents on
  *                entry do not matter; must not be used by anything else until the work
  *                queued on `stream` by this call has finished

@@ -42,7 +42,9 @@ def _gpu_q(hqq, packed, scale, zero, rows, cols, nbits, g, axis):
 # fast path: axis 1, 2/4 bit, cols and g multiples of the codes per word; the rest generic
 LAYOUTS = [(4, 64, 1, 96, 512), (2, 16, 1, 64, 256), (4, 128, 1, 33, 1024), (2, 64, 1, 17, 320),
            (3, 64, 1, 40, 640), (3, 10, 1, 21, 130), (4, 64, 0, 64, 192), (2, 16, 0, 48, 80),
-           (4, 3, 1, 30, 21), (4, 24, 1, 12, 96)]
+           (4, 3, 1, 30, 21), (4, 24, 1, 12, 96),
+           # one word per row, a ragged last CTA of rows, the largest group, one row
+           (4, 8, 1, 7, 8), (2, 16, 1, 1, 16), (4, 256, 1, 9, 4096), (2, 256, 1, 3, 8192)]
 
 
 @pytest.mark.parametrize("nbits,g,axis,rows,cols", LAYOUTS, ids=lambda v: str(v))
@@ -59,6 +61,21 @@ def test_gemv_random_codes(hqq, nbits, g, axis, rows, cols):
     q = _gpu_q(hqq, packed, scale, zero, rows, cols, nbits, g, axis)
     y = hqq.hqq_gemv(q, torch.from_numpy(x).cuda()).cpu().numpy()
     _check(y, ref, mag, cols, (nbits, g, axis, rows, cols))
+
+
+def test_gemv_large_x(hqq):
+    # x near the fp16 range: products up to ~1e5, still exact in binary32 before the sum
+    rows, cols, nbits, g = 24, 512, 4, 64
+    r = np.random.default_rng(13)
+    packed = oracle.pack(r.integers(0, 16, rows * cols).astype(np.uint8), nbits)
+    G = rows * cols // g
+    scale = (r.random(G) * 0.05 + 1e-3).astype(np.float16)
+    zero = (r.random(G) * 16).astype(np.float16)
+    x = (r.standard_normal(cols) * 2e4).clip(-6e4, 6e4).astype(np.float16)
+    ref, mag = oracle.gemv(packed, scale, zero, rows, cols, nbits, g, 1, x)
+    q = _gpu_q(hqq, packed, scale, zero, rows, cols, nbits, g, 1)
+    y = hqq.hqq_gemv(q, torch.from_numpy(x).cuda()).cpu().numpy()
+    _check(y, ref, mag, cols, "large x")
 
 
 def test_gemv_unaligned_x_takes_the_generic_path(hqq):

@@ -58,8 +58,21 @@ def _tiny_range(rows, cols, seed):
     return W.astype(np.float16)
 
 
+def _negative(rows, cols, seed):
+    # every group entirely negative and far from 0: z0 = -min*s is large and positive
+    r = np.random.default_rng(seed)
+    return (-1000.0 - 24.0 * r.random((rows, cols))).astype(np.float16)
+
+
+def _positive(rows, cols, seed):
+    # every group entirely positive, offset per row: z0 is large and negative
+    r = np.random.default_rng(seed)
+    base = r.uniform(0.5, 600.0, (rows, 1))
+    return (base + r.standard_normal((rows, cols)) * 0.01 * base).astype(np.float16)
+
+
 GENS = {"t": wl.student_t, "n": wl.outlier_normal, "bimodal": _bimodal, "sparse": _sparse,
-        "wide": _wide, "const": _const, "tiny": _tiny_range}
+        "wide": _wide, "const": _const, "tiny": _tiny_range, "neg": _negative, "pos": _positive}
 
 # rows, cols, nbits, group_size, axis, iters, generator
 EDGE = [
@@ -91,6 +104,10 @@ EDGE = [
     (40, 41, 3, 8, 0, 20, "t"),           # axis 0, G = 205, odd
     (64, 256, 4, 64, 0, 20, "bimodal"),
     (64, 256, 4, 64, 0, 20, "wide"),
+    (64, 256, 4, 64, 1, 20, "neg"),       # one-signed groups far from 0: large |z|
+    (64, 256, 2, 16, 1, 20, "pos"),
+    (64, 256, 3, 64, 1, 20, "neg"),
+    (64, 256, 4, 64, 0, 20, "pos"),
 ]
 
 

@@ -166,6 +166,15 @@ class ClockSampler:
                 "window": window, "power_w_max": max((num(p[3]) or 0.0) for p in win)}
 
 
+def launches_per_step(nbits: int, group: int, axis: int, n: int) -> int:
+    """Kernels one quantize + dequantize step launches: the zero kernel, the stream or search
+    kernel and the fixup kernel, a pack kernel when an axis-0 layout's groups do not fill
+    whole packed words, and the dequant kernel."""
+    cpw = {2: 16, 3: 10, 4: 8}[nbits]
+    pack = axis == 0 and (n // group) % cpw != 0
+    return 4 + (1 if pack else 0)
+
+
 def shard(items, rank: int, ws: int):
     """This rank's share of independent work items (every item on exactly one rank)."""
     return items[rank::ws]
@@ -330,7 +339,7 @@ def run_stack(args, ws, rank, local):
                          "achieved": ach, "peak": alu_peak, "unit": "Tops/s", "frac": ach / alu_peak,
                          "traffic": None, "alg_ops_per_step": alg_ops * ws},
             "e2e": None,
-            "gpu_launches": 3 * len(Ws) * args.steps,
+            "gpu_launches": launches_per_step(NBITS, GROUP, AXIS, 4096 * 4096) * len(Ws) * args.steps,
             "clocks": clocks,
         }
         if not args.no_cpu_baseline:
@@ -594,7 +603,7 @@ def main():
             "e2e": {"value": ws * N / (e2e_ms / 1e3) / 1e9, "unit": UNIT,
                     "h2d_bytes_per_step": 2 * N,
                     "d2h_bytes_per_step": packed_bytes + 4 * G + 2 * N},
-            "gpu_launches": 3 * K,
+            "gpu_launches": launches_per_step(NBITS, GROUP, AXIS, N) * K,
             "clocks": clocks,
         }
         if not args.no_cpu_baseline:

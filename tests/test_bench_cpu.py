@@ -41,3 +41,9 @@ def test_profiled_traffic_only_while_the_code_matches(tmp_path, monkeypatch):
     src.write_text(SRC.replace("1.0f", "3.0f"))
     assert bench.profiled_traffic() is None
 
+
+
+def test_launch_count_per_step():
+    assert bench.launches_per_step(4, 64, 1, 4096 * 4096) == 4      # zero, stream, fixup, dequant
+    assert bench.launches_per_step(4, 128, 0, 4096 * 4096) == 4     # G = 131072 fills words
+    assert bench.launches_per_step(4, 16, 0, 30 * 32) == 5          # G = 60: byte staging + pack

@@ -1,15 +1,26 @@
-"""Benchmark: HQQ quantize+pack and dequantize of a 4096x4096 fp16 weight on B200.
+"""Benchmark: HQQ quantize+pack and dequantize on B200.
 
 One step = the whole hot path over one matrix: hqq_quantize (min-max init, proximal rounds
 with the tensor-wide stop rule, final quantize, bit-packing, fp16 metadata) followed by
-hqq_dequantize.  Inputs rotate over R copies so that every step reads its matrix from HBM
-(R * 33.5 MB > 126 MB of L2).  Prints one JSON line (rank 0).
+hqq_dequantize.  Inputs rotate over enough copies that every step reads its matrix from HBM
+(more than twice the 126 MB L2).  Rank 0 prints one JSON line:
+  - `value`: quantize+pack Gweights/s (all ranks' weights over the max-over-ranks time);
+  - `roofline`: the quantize call against the ALU issue peak, with the stream kernel's DRAM
+    traffic from the committed ncu summary while its code is unchanged;
+  - `e2e`: the same metric through the public API with pinned host buffers, copies included;
+  - `cpu_baseline`: the CPU oracle on the host;
+  - `dequant_back_to_back` and `gemv`: dequantize and the fused forward product, each timed
+    back to back by CUDA-graph replay, with the unfused dequantize + matmul beside the latter.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                  [--workload attn|small|mlp_b2|mlp_b3|attn_ax0|stack]
 
---impl reference times the CPU oracle (the plain C reference of the method) on the host on a
-bounded slice of the same workload.  Under torchrun every rank quantizes its own matrices (no
-data-path communication: weak scaling); the reference arm runs on rank 0 only.
+--workload picks the configuration: attn, the default, is the 4096x4096 4-bit group-64
+headline; stack quantizes and dequantizes all 224 matrices of the 7B-like stack per step.
+--impl reference times the CPU oracle (the plain C reference of the method) on the host on
+bounded slices of the same workload.  Under torchrun every rank quantizes its own matrices,
+with no data-path communication (weak scaling; stack: the matrices are split, strong scaling).
+The reference arm runs on rank 0 only.
 """
 from __future__ import annotations
 

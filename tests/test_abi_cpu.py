@@ -137,3 +137,13 @@ def test_gemv_rejects_on_host(L):
     assert call(pk=FAKE + 4) == 2          # packed not 16-byte aligned
     assert call(x=FAKE + 1) == 2
     assert call(y=FAKE + 2) == 2
+
+
+def test_binding_arity_matches_the_header():
+    # every prototype's parameter count equals the binding's ctypes argtypes
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    protos = dict(re.findall(r"\b(hqq_[a-z_0-9]+)\s*\(([^)]*)\)\s*;", text))
+    assert set(protos) == set(hqq.SIGNATURES)
+    for name, params in protos.items():
+        n = 0 if params.strip() in ("", "void") else params.count(",") + 1
+        assert n == len(hqq.SIGNATURES[name][1]), (name, n, len(hqq.SIGNATURES[name][1]))

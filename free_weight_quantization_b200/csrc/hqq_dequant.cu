@@ -1,0 +1,356 @@
+// hqq_dequant.cu -- unpack + dequantize and the fused forward product of the B200 HQQ library
+// [HQQ 算法解读, "量化公式" and "从压缩文件到一次前向"].
+#include "hqq_common.cuh"
+
+namespace {
+
+// ------------------------------------------------------------------------------------------
+// dequantize [HQQ 算法解读, "量化公式" and "从压缩文件到一次前向"]: W = (q - z) * Delta
+// One packed 32-bit word (8, 16 or 10 codes) per lane and step, so that a warp's loads cover
+// 128 contiguous bytes and its stores 512 contiguous bytes (4 bit).  A thread handles kDqU
+// words spaced a block apart, all loaded before any is expanded.
+//   MODE 0: axis 1, group_size a multiple of the codes per word: one group per word
+//   MODE 1: axis 1, any group size
+//   MODE 2: axis 0 (element n belongs to group n % G)
+// ------------------------------------------------------------------------------------------
+constexpr int kDqU = 4;
+constexpr int kDqThreads = 256;
+
+template <int NB, int MODE>
+__global__ void __launch_bounds__(kDqThreads) hqq_dequant_kernel(
+    const uint32_t *__restrict__ packed, const __half *__restrict__ scale,
+    const __half *__restrict__ zero, int64_t N, int g, int64_t G, int64_t packed_bytes,
+    int wpg_shift, bool vec_meta, __half *__restrict__ out) {
+    constexpr int CPW = Pack<NB>::cpw;
+    constexpr uint32_t MASK = (1u << NB) - 1u;
+    const int64_t nwords = (N + CPW - 1) / CPW;
+    const int64_t wbase = (int64_t)blockIdx.x * (kDqThreads * kDqU) + threadIdx.x;
+    wait_prerequisite();  // the codes may come from the kernel launched just before
+    allow_dependents();
+    uint32_t wd[kDqU];
+    // MODE 3 (axis 1, g >= codes per word): a word spans at most two groups; both metadata
+    // pairs are loaded here, alongside the word, and codes c < cb belong to the first
+    float z0[MODE == 3 ? kDqU : 1], d0[MODE == 3 ? kDqU : 1], z1[MODE == 3 ? kDqU : 1],
+        d1[MODE == 3 ? kDqU : 1];
+    int cb[MODE == 3 ? kDqU : 1];
+#pragma unroll
+    for (int u = 0; u < kDqU; ++u) {
+        const int64_t wi = wbase + u * kDqThreads;
+        wd[u] = 0;
+        if (wi < nwords) {
+            if (wi * 4 + 4 <= packed_bytes) {
+                wd[u] = __ldcs(packed + wi);
+            } else {  // the last word of a byte-sized packing may be short
+                const uint8_t *pb = reinterpret_cast<const uint8_t *>(packed);
+                for (int b = 0; b < 4 && wi * 4 + b < packed_bytes; ++b)
+                    wd[u] |= (uint32_t)pb[wi * 4 + b] << (8 * b);
+            }
+            if constexpr (MODE == 3) {
+                const int64_t n0 = wi * CPW;
+                const int64_t k0 = wpg_shift >= 0 ? (n0 >> wpg_shift) : n0 / g;
+                const int64_t k1 = k0 + 1 < G ? k0 + 1 : k0;
+                cb[u] = (int)(g - (n0 - k0 * g));
+                z0[u] = __half2float(__ldg(zero + k0));
+                d0[u] = __half2float(__ldg(scale + k0));
+                z1[u] = __half2float(__ldg(zero + k1));
+                d1[u] = __half2float(__ldg(scale + k1));
+            }
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < kDqU; ++u) {
+        const int64_t wi = wbase + u * kDqThreads;
+        if (wi >= nwords) break;
+        const int64_t n0 = wi * CPW;
+        uint32_t res[(CPW + 1) / 2];
+        float v[CPW];
+        if constexpr (MODE == 3) {
+#pragma unroll
+            for (int c = 0; c < CPW; ++c) {
+                const bool first = c < cb[u];
+                const float qf = __fsub_rn(__int_as_float(0x4B000000 | (int)((wd[u] >> (NB * c)) & MASK)), 8388608.0f);
+                v[c] = __fmul_rn(__fsub_rn(qf, first ? z0[u] : z1[u]), first ? d0[u] : d1[u]);
+            }
+        } else if (MODE == 0) {
+            const int64_t k = wpg_shift >= 0 ? (wi >> wpg_shift) : (n0 / g);
+            const float zf = __half2float(zero[k]), df = __half2float(scale[k]);
+#pragma unroll
+            for (int c = 0; c < CPW; ++c) {
+                const float qf = __fsub_rn(__int_as_float(0x4B000000 | (int)((wd[u] >> (NB * c)) & MASK)), 8388608.0f);
+                v[c] = __fmul_rn(__fsub_rn(qf, zf), df);
+            }
+        } else if (MODE == 2 && vec_meta) {
+            // CPW consecutive groups starting at a multiple of 8: 16-byte metadata loads
+            const int64_t k0 = n0 % G;
+#pragma unroll
+            for (int c8 = 0; c8 < CPW; c8 += 8) {
+                const uint4 zv = __ldg(reinterpret_cast<const uint4 *>(zero + k0 + c8));
+                const uint4 dv = __ldg(reinterpret_cast<const uint4 *>(scale + k0 + c8));
+                const __half *zh = reinterpret_cast<const __half *>(&zv);
+                const __half *dh = reinterpret_cast<const __half *>(&dv);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const float qf = __fsub_rn(__int_as_float(0x4B000000 | (int)((wd[u] >> (NB * (c8 + c))) & MASK)), 8388608.0f);
+                    v[c8 + c] = __fmul_rn(__fsub_rn(qf, __half2float(zh[c])), __half2float(dh[c]));
+                }
+            }
+        } else {
+            int64_t k;
+            int j = 0;
+            if (MODE == 1) {
+                k = n0 / g;
+                j = (int)(n0 - k * g);
+            } else {
+                k = n0 % G;
+            }
+            float zf = __half2float(zero[k]), df = __half2float(scale[k]);
+#pragma unroll
+            for (int c = 0; c < CPW; ++c) {
+                const float qf = __fsub_rn(__int_as_float(0x4B000000 | (int)((wd[u] >> (NB * c)) & MASK)), 8388608.0f);
+                v[c] = __fmul_rn(__fsub_rn(qf, zf), df);
+                if (c + 1 < CPW && n0 + c + 1 < N) {  // move to the group of the next element
+                    if (MODE == 1) {
+                        if (++j == g) {
+                            j = 0;
+                            ++k;
+                            zf = __half2float(zero[k]);
+                            df = __half2float(scale[k]);
+                        }
+                    } else {
+                        if (++k == G) k = 0;
+                        zf = __half2float(zero[k]);
+                        df = __half2float(scale[k]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < CPW; c += 2) {
+            const __half2 h2 = __floats2half2_rn(v[c], c + 1 < CPW ? v[c + 1] : 0.0f);
+            memcpy(&res[c / 2], &h2, 4);
+        }
+        if (n0 + CPW <= N) {
+            if (CPW % 8 == 0) {  // 16 or 32 bytes per word, 16-byte aligned
+                uint4 *dst = reinterpret_cast<uint4 *>(out + n0);
+#pragma unroll
+                for (int i = 0; i < CPW / 8; ++i)
+                    __stcs(dst + i, make_uint4(res[4 * i], res[4 * i + 1], res[4 * i + 2], res[4 * i + 3]));
+            } else {  // 10 codes: 20 bytes, 4-byte aligned
+                uint32_t *dst = reinterpret_cast<uint32_t *>(out + n0);
+#pragma unroll
+                for (int i = 0; i < CPW / 2; ++i) __stcs(dst + i, res[i]);
+            }
+        } else {
+            unsigned short *o16 = reinterpret_cast<unsigned short *>(out + n0);
+#pragma unroll
+            for (int c = 0; c < CPW; ++c)
+                if (n0 + c < N) o16[c] = (unsigned short)(res[c / 2] >> (16 * (c % 2)));
+        }
+    }
+}
+
+template <int NB>
+cudaError_t launch_dequant(const uint8_t *pk, const __half *sc, const __half *ze, int64_t N, int g,
+                    int64_t G, int axis, int64_t pb, __half *out, cudaStream_t st) {
+    constexpr int CPW = Pack<NB>::cpw;
+    const int64_t nwords = (N + CPW - 1) / CPW;
+    const unsigned blocks = (unsigned)((nwords + kDqThreads * kDqU - 1) / (kDqThreads * kDqU));
+    const uint32_t *pw = reinterpret_cast<const uint32_t *>(pk);
+    int shift = -1;
+    if (g % CPW == 0) {
+        const int wpg = g / CPW;
+        if ((wpg & (wpg - 1)) == 0) { shift = 0; while ((1 << shift) < wpg) ++shift; }
+    }
+    const bool vec_meta = CPW % 8 == 0 && G % 8 == 0 && (((uintptr_t)sc | (uintptr_t)ze) & 15) == 0;
+    // programmatic launch: overlaps the kernel before it, which the kernel waits for
+    if (axis == 1 && g % CPW == 0)
+        return launch_pdl(hqq_dequant_kernel<NB, 0>, blocks, kDqThreads, 0, st, pw, sc, ze, N, g, G, pb, shift, false, out);
+    if (axis == 1 && g >= CPW) {  // a word spans at most two groups
+        int gs = -1;
+        if ((g & (g - 1)) == 0) { gs = 0; while ((1 << gs) < g) ++gs; }
+        return launch_pdl(hqq_dequant_kernel<NB, 3>, blocks, kDqThreads, 0, st, pw, sc, ze, N, g, G, pb, gs, false, out);
+    }
+    if (axis == 1)
+        return launch_pdl(hqq_dequant_kernel<NB, 1>, blocks, kDqThreads, 0, st, pw, sc, ze, N, g, G, pb, -1, false, out);
+    return launch_pdl(hqq_dequant_kernel<NB, 2>, blocks, kDqThreads, 0, st, pw, sc, ze, N, g, G, pb, -1, vec_meta, out);
+}
+
+// ==========================================================================================
+// The quantized layer's forward product for one input vector [HQQ 算法解读,
+// "从压缩文件到一次前向"]: unpack -> (q - zero) * scale -> x @ W_hat.T, fused so that W_hat never
+// reaches memory.  Each W_hat[r, c] is the exact fp16 value hqq_dequantize writes; the product
+// with the fp16 x[c] is exact in binary32, and the row sum runs in binary32.
+// ==========================================================================================
+
+// Axis 1, 2- or 4-bit, cols and g multiples of the codes per word: one warp per output row.
+// Lane l takes the row's words l, l + 32, ... (every warp load covers 128 contiguous bytes) and
+// loads kGvU of them, with their metadata, before using any: a 4096-column 4-bit row is one
+// batch, so a warp waits for memory once.  A word's codes are dequantized in pairs exactly as
+// hqq_dequantize does (a code c becomes 2^23 + c by a byte permute against 0x4B000000, then
+// (q - z) * Delta in binary32, rounded to fp16) and multiplied with x in packed binary32 FMAs.
+constexpr int kGvU = 16;
+
+template <int NB>
+__device__ __forceinline__ float2 gemv_word(uint32_t w, float zf, float df, const __half *xw,
+                                            float2 acc) {
+    const float2 nm = make_float2(-8388608.0f, -8388608.0f), nz = make_float2(-zf, -zf);
+    const float2 d2 = make_float2(df, df);
+    constexpr int CPW = Pack<NB>::cpw;
+    uint32_t xs[CPW / 2];
+#pragma unroll
+    for (int v = 0; v < CPW / 8; ++v) {
+        const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(xw) + v);
+        xs[4 * v] = xv.x; xs[4 * v + 1] = xv.y; xs[4 * v + 2] = xv.z; xs[4 * v + 3] = xv.w;
+    }
+    if constexpr (NB == 4) {
+        const uint32_t ev = w & 0x0F0F0F0Fu, od = (w >> 4) & 0x0F0F0F0Fu;  // codes 2i, 2i+1 in byte i
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 q = make_float2(__uint_as_float(__byte_perm(ev, 0x4B000000u, 0x7540u + i)),
+                                         __uint_as_float(__byte_perm(od, 0x4B000000u, 0x7540u + i)));
+            const float2 v = __fmul2_rn(__fadd2_rn(__fadd2_rn(q, nm), nz), d2);
+            const float2 xf = __half22float2(*reinterpret_cast<const __half2 *>(&xs[i]));
+            acc = __ffma2_rn(__half22float2(__floats2half2_rn(v.x, v.y)), xf, acc);
+        }
+    } else {  // 2 bit: field s of byte b is code 4b + s
+        uint32_t f[4];
+#pragma unroll
+        for (int s = 0; s < 4; ++s) f[s] = (w >> (2 * s)) & 0x03030303u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {  // codes 2i, 2i+1: byte i/2, fields 2(i%2) and +1
+            const int b = i >> 1, s = 2 * (i & 1);
+            const float2 q = make_float2(__uint_as_float(__byte_perm(f[s], 0x4B000000u, 0x7540u + b)),
+                                         __uint_as_float(__byte_perm(f[s + 1], 0x4B000000u, 0x7540u + b)));
+            const float2 v = __fmul2_rn(__fadd2_rn(__fadd2_rn(q, nm), nz), d2);
+            const float2 xf = __half22float2(*reinterpret_cast<const __half2 *>(&xs[i]));
+            acc = __ffma2_rn(__half22float2(__floats2half2_rn(v.x, v.y)), xf, acc);
+        }
+    }
+    return acc;
+}
+
+template <int NB>
+__global__ void __launch_bounds__(256) hqq_gemv_kernel(const uint32_t *__restrict__ packed,
+                                                       const __half *__restrict__ scale,
+                                                       const __half *__restrict__ zero,
+                                                       int64_t rows, int wpr, int gpr,
+                                                       int wpg_shift, int wpg,
+                                                       const __half *__restrict__ x,
+                                                       float *__restrict__ y) {
+    constexpr int CPW = Pack<NB>::cpw;
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    wait_prerequisite();  // codes and x may come from the kernel launched just before
+    allow_dependents();
+    if (row >= rows) return;  // whole warps
+    const uint32_t *prow = packed + row * wpr;
+    const int64_t k0 = row * gpr;
+    float2 acc = make_float2(0.0f, 0.0f);
+    for (int w0 = lane; w0 < wpr; w0 += 32 * kGvU) {
+        uint32_t wd[kGvU];
+        float zf[kGvU], df[kGvU];
+#pragma unroll
+        for (int u = 0; u < kGvU; ++u) {
+            const int w = w0 + 32 * u;
+            wd[u] = 0;
+            zf[u] = 0.0f;
+            df[u] = 0.0f;
+            if (w < wpr) {
+                const int64_t k = k0 + (wpg_shift >= 0 ? (w >> wpg_shift) : w / wpg);
+                wd[u] = __ldcs(prow + w);
+                zf[u] = __half2float(__ldg(zero + k));
+                df[u] = __half2float(__ldg(scale + k));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kGvU; ++u) {
+            const int w = w0 + 32 * u;
+            if (w < wpr) acc = gemv_word<NB>(wd[u], zf[u], df[u], x + (int64_t)w * CPW, acc);
+        }
+    }
+    float s = __fadd_rn(acc.x, acc.y);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s = __fadd_rn(s, __shfl_xor_sync(kFull, s, off));
+    if (lane == 0) y[row] = s;
+}
+
+// Any other layout: one warp per output row, each lane takes columns lane, lane + 32, ...
+// and reads its codes one at a time (flat row-major code order, groups by axis).
+template <int NB>
+__global__ void __launch_bounds__(256) hqq_gemv_any_kernel(const uint8_t *__restrict__ packed,
+                                                           const __half *__restrict__ scale,
+                                                           const __half *__restrict__ zero,
+                                                           int64_t rows, int64_t cols, int64_t g,
+                                                           int64_t G, int axis,
+                                                           const __half *__restrict__ x,
+                                                           float *__restrict__ y) {
+    constexpr uint32_t MASK = (1u << NB) - 1u;
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    wait_prerequisite();
+    allow_dependents();
+    if (row >= rows) return;
+    float acc = 0.0f;
+    for (int64_t c = lane; c < cols; c += 32) {
+        const int64_t n = row * cols + c;
+        uint32_t q;
+        if (NB == 3) {
+            const uint32_t wv = __ldg(reinterpret_cast<const uint32_t *>(packed) + n / 10);
+            q = (wv >> (3 * (int)(n % 10))) & MASK;
+        } else {
+            const int per = 8 / NB;
+            q = ((uint32_t)__ldg(packed + n / per) >> (NB * (int)(n % per))) & MASK;
+        }
+        const int64_t k = axis == 1 ? n / g : n % G;
+        const float v = __fmul_rn(__fsub_rn((float)q, __half2float(__ldg(zero + k))), __half2float(__ldg(scale + k)));
+        acc = __fmaf_rn(__half2float(__float2half_rn(v)), __half2float(__ldg(x + c)), acc);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(kFull, acc, off));
+    if (lane == 0) y[row] = acc;
+}
+
+template <int NB>
+cudaError_t launch_gemv_nb(const uint8_t *pk, const __half *sc, const __half *ze, int64_t rows,
+                        int64_t cols, int64_t g, int64_t G, int axis, const __half *x, float *y,
+                        cudaStream_t st) {
+    constexpr int CPW = Pack<NB>::cpw;
+    const unsigned blocks = (unsigned)((rows + 7) / 8);
+    const int64_t wpr = cols / CPW;
+    if (NB != 3 && axis == 1 && cols % CPW == 0 && g % CPW == 0 && ((uintptr_t)x & 15) == 0 &&
+        wpr < ((int64_t)1 << 30)) {
+        const int wpg = (int)(g / CPW);
+        int shift = -1;
+        if ((wpg & (wpg - 1)) == 0) { shift = 0; while ((1 << shift) < wpg) ++shift; }
+        return launch_pdl(hqq_gemv_kernel<NB>, blocks, 256, 0, st, (const uint32_t *)pk, sc, ze,
+                          rows, (int)wpr, (int)(cols / g), shift, wpg, x, y);
+    }
+    return launch_pdl(hqq_gemv_any_kernel<NB>, blocks, 256, 0, st, pk, sc, ze, rows, cols, g, G,
+                      axis, x, y);
+}
+
+}  // namespace
+
+namespace hqq_impl {
+
+cudaError_t launch_dequantize(int nbits, const uint8_t *pk, const __half *sc, const __half *ze,
+                              int64_t N, int g, int64_t G, int axis, int64_t pb, __half *out,
+                              cudaStream_t st) {
+    switch (nbits) {
+    case 4: return launch_dequant<4>(pk, sc, ze, N, g, G, axis, pb, out, st);
+    case 3: return launch_dequant<3>(pk, sc, ze, N, g, G, axis, pb, out, st);
+    default: return launch_dequant<2>(pk, sc, ze, N, g, G, axis, pb, out, st);
+    }
+}
+
+cudaError_t launch_gemv(int nbits, const uint8_t *pk, const __half *sc, const __half *ze,
+                        int64_t rows, int64_t cols, int64_t g, int64_t G, int axis,
+                        const __half *x, float *y, cudaStream_t st) {
+    switch (nbits) {
+    case 4: return launch_gemv_nb<4>(pk, sc, ze, rows, cols, g, G, axis, x, y, st);
+    case 3: return launch_gemv_nb<3>(pk, sc, ze, rows, cols, g, G, axis, x, y, st);
+    default: return launch_gemv_nb<2>(pk, sc, ze, rows, cols, g, G, axis, x, y, st);
+    }
+}
+
+}  // namespace hqq_impl

@@ -56,7 +56,9 @@ def test_packed_bytes_rejects(L):
 def test_workspace_bytes(L):
     ws = hqq.hqq_quantize_workspace_bytes
     assert ws(4096, 4096, 4, 64, 1, 20) > 0
-    assert ws(4096, 4096, 4, 64, 1, 20) < 4096 * 4096 // 16  # small: round sums + 1 byte/group
+    # small: round sums + 1 byte per group (its last round)
+    G = 4096 * 4096 // 64
+    assert G <= ws(4096, 4096, 4, 64, 1, 20) < G + 65536
     assert ws(10, 10, 4, 3, 1, 20) == 0        # 100 % 3 != 0
     assert ws(16, 16, 5, 16, 1, 20) == 0       # 5 bits
     assert ws(16, 16, 4, 16, 2, 20) == 0       # axis 2

@@ -19,12 +19,26 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "hqq_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "libhqq_oracle.so")
+# The all-core timing build: the same source with its round loop spread over OpenMP threads
+# (bench.py's CPU baseline only; every test uses the single-threaded build).
+_LIB_PAR_PATH = os.path.join(_HERE, "libhqq_oracle_omp.so")
 # Test hook: the mutation test points this at a deliberately broken build of the oracle.
 _LIB_OVERRIDE = os.environ.get("HQO_LIB_OVERRIDE")
 # No contraction of a*b+c into fma, no fast-math: every binary32 operation rounds once.
 CFLAGS = ["-O2", "-std=gnu11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
 
 _lib = None
+_lib_par = None
+
+
+def build_parallel(force: bool = False) -> str:
+    """Compile the all-core timing build of hqq_oracle.c (OpenMP over groups, exact integer
+    reduction of each round's error) into oracle/libhqq_oracle_omp.so."""
+    if force or not os.path.exists(_LIB_PAR_PATH) or os.path.getmtime(_LIB_PAR_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PAR_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *CFLAGS, "-fopenmp", "-DHQO_PARALLEL", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB_PAR_PATH)
+    return _LIB_PAR_PATH
 
 
 def build(force: bool = False) -> str:
@@ -38,11 +52,18 @@ def build(force: bool = False) -> str:
     return _LIB_PATH
 
 
-def _load():
-    global _lib
-    if _lib is not None:
-        return _lib
-    lib = ctypes.CDLL(build())
+def _load(parallel: bool = False):
+    global _lib, _lib_par
+    if parallel:
+        if _lib_par is None:
+            _lib_par = _declare(ctypes.CDLL(build_parallel()))
+        return _lib_par
+    if _lib is None:
+        _lib = _declare(ctypes.CDLL(build()))
+    return _lib
+
+
+def _declare(lib):
     P = ctypes.c_void_p
     i64, i32, f32, f64 = ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_double
     lib.hqo_half_to_float.argtypes = [ctypes.c_uint16]
@@ -71,7 +92,6 @@ def _load():
     lib.hqo_dequant.argtypes = [P, P, P, i64, i64, i32, i64, i32, P]
     lib.hqo_gemv.argtypes = [P, P, P, i64, i64, i32, i64, i32, P, P, P]
     lib.hqo_dequant.restype = i32
-    _lib = lib
     return lib
 
 
@@ -151,11 +171,12 @@ DEFAULTS = dict(iters=20, lp_norm=0.7, beta=10.0, kappa=1.01, eps_tiny=1e-4, sca
 
 def quantize(W, nbits: int, group_size: int, axis: int = 1, iters: int = 20, lp_norm: float = 0.7,
              beta: float = 10.0, kappa: float = 1.01, eps_tiny: float = 1e-4,
-             scale_max: float = 2e4) -> dict:
+             scale_max: float = 2e4, parallel: bool = False) -> dict:
     """HQQ quantize+pack of a 2-D fp16 matrix.  Returns a dict with codes (flat, one per
     byte), s, z (binary32 per group; z is the kept zero), scale/zero (fp16 Delta = 1/s and z),
     packed bytes, iters_run, err_trace (exact per-iteration error sums, units of 2^-32, as
-    Python ints) and mae_trace."""
+    Python ints) and mae_trace.  parallel=True runs the all-core timing build (same results;
+    for the benchmark's CPU baseline)."""
     Wu = _as_u16(W)
     assert Wu.ndim == 2
     rows, cols = Wu.shape
@@ -169,7 +190,7 @@ def quantize(W, nbits: int, group_size: int, axis: int = 1, iters: int = 20, lp_
     run = ctypes.c_int(0)
     trace = np.zeros(max(2 * iters, 2), np.uint64)
     mae = np.zeros(max(iters, 1), np.float64)
-    rc = _load().hqo_quantize(_ptr(Wu), rows, cols, nbits, group_size, axis, iters, lp_norm, beta,
+    rc = _load(parallel).hqo_quantize(_ptr(Wu), rows, cols, nbits, group_size, axis, iters, lp_norm, beta,
                               kappa, eps_tiny, scale_max, _ptr(codes), _ptr(s), _ptr(z),
                               ctypes.byref(run), _ptr(trace), _ptr(mae))
     if rc != 0:

@@ -241,12 +241,31 @@ int hqo_quantize(const uint16_t *W, int64_t rows, int64_t cols, int nbits, int64
     double beta = beta0;
     for (int i = 0; i < iters; i++) {
         unsigned __int128 total = 0;
+#ifdef HQO_PARALLEL
+        /* Timing build only (the all-core CPU baseline of the benchmark): the same group
+           passes, spread over threads; each thread adds its groups' exact integer errors and
+           the partial sums are added afterwards, which gives the same total in any order. */
+#pragma omp parallel
+        {
+            unsigned __int128 part = 0;
+#pragma omp for schedule(static)
+            for (int64_t k = 0; k < G; k++) {
+                float err;
+                hqo_group_pass(wg + k * g, g, nbits, s_out[k], z[k], beta, lp_norm, NULL, &err,
+                               &znext[k]);
+                part += err_fixed(err);
+            }
+#pragma omp critical
+            total += part;
+        }
+#else
         for (int64_t k = 0; k < G; k++) {
             float err;
             hqo_group_pass(wg + k * g, g, nbits, s_out[k], z[k], beta, lp_norm, NULL, &err,
                            &znext[k]);
             total += err_fixed(err);
         }
+#endif
         run = i + 1;
         if (err_trace) {
             err_trace[2 * i] = (uint64_t)total;

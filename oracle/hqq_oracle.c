@@ -22,7 +22,8 @@
  *                       when the reconstruction MAE is not better than the best so far;
  *                       quantize once more with the original W
  *   packing ........... [HQQ 算法解读, "为什么一定要分组"] two 4-bit codes per byte, four 2-bit
- *                       codes per byte, ten 3-bit codes per 32-bit word
+ *                       codes per byte, ten 3-bit codes per 32-bit word; 5- and 6-bit codes one
+ *                       per byte
  *   forward product ... [HQQ 算法解读, "从压缩文件到一次前向"] unpack -> (q - zero)*scale ->
  *                       x @ W_hat.T (hqo_gemv, one input vector)
  *
@@ -48,7 +49,9 @@
  *     from (z_i); when iteration i is accepted z_i becomes the kept zero; the kept zero
  *     after the loop is the one whose MAE was best (never an unmeasured z);
  *   - codes are packed in flat row-major order for both axes, lowest index in the
- *     lowest bits; the tail of the last byte or word is zero.
+ *     lowest bits; the tail of the last byte or word is zero;
+ *   - 7- and 8-bit codes are stored one per byte like 5 and 6 bits; 1-bit codes, which the
+ *     pages name only in passing, are packed eight per byte like the 2- and 4-bit codes.
  */
 #include <math.h>
 #include <stdint.h>
@@ -304,14 +307,17 @@ void hqo_metadata(const float *s, const float *z, int64_t G, uint16_t *scale_h, 
     }
 }
 
-/* Packed size in bytes [HQQ 算法解读, "为什么一定要分组"]. */
+/* Packed size in bytes [HQQ 算法解读, "为什么一定要分组"]: 4 bit two codes per byte, 2 bit four,
+ * 3 bit ten per 32-bit word; 5 and 6 bit are stored one code per byte, and so are 7 and 8 bit;
+ * 1 bit (which the pages name without a layout) eight codes per byte. */
 int64_t hqo_packed_bytes(int64_t n, int nbits)
 {
     switch (nbits) {
     case 4: return (n + 1) / 2;
     case 2: return (n + 3) / 4;
+    case 1: return (n + 7) / 8;
     case 3: return 4 * ((n + 9) / 10);
-    default: return n;                     /* 5..8 bits and 1 bit: one code per byte */
+    default: return n;                     /* 5..8 bits: one code per byte */
     }
 }
 
@@ -320,7 +326,7 @@ void hqo_pack(const uint8_t *codes, int64_t n, int nbits, uint8_t *packed)
 {
     int64_t nb = hqo_packed_bytes(n, nbits);
     memset(packed, 0, (size_t)nb);
-    if (nbits == 4 || nbits == 2) {
+    if (nbits == 4 || nbits == 2 || nbits == 1) {
         int per = 8 / nbits;
         for (int64_t i = 0; i < n; i++)
             packed[i / per] |= (uint8_t)(codes[i] << (nbits * (i % per)));
@@ -338,7 +344,7 @@ void hqo_pack(const uint8_t *codes, int64_t n, int nbits, uint8_t *packed)
 
 void hqo_unpack(const uint8_t *packed, int64_t n, int nbits, uint8_t *codes)
 {
-    if (nbits == 4 || nbits == 2) {
+    if (nbits == 4 || nbits == 2 || nbits == 1) {
         int per = 8 / nbits;
         for (int64_t i = 0; i < n; i++)
             codes[i] = (uint8_t)((packed[i / per] >> (nbits * (i % per))) & ((1 << nbits) - 1));

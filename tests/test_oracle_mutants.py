@@ -34,6 +34,7 @@ MUTANTS = {
                           "memcpy(z_out, znext, sizeof(float) * (size_t)G);   /* z_i"),
     "beta not updated": ("beta = beta * kappa;", ""),
     "axis0 index": ("return axis == 1 ? k * g + j : j * G + k;", "return axis == 1 ? k * g + j : k * g + j;"),
+    "1-bit one per byte": ("case 1: return (n + 7) / 8;", "case 1: return n;"),
     "nibble order": ("packed[i / per] |= (uint8_t)(codes[i] << (nbits * (i % per)));",
                      "packed[i / per] |= (uint8_t)(codes[i] << (nbits * (per - 1 - i % per)));"),
     "dequant group index": ("int64_t k = axis == 1 ? n / g : n % G;", "int64_t k = axis == 1 ? n / g : n / g;"),

@@ -110,7 +110,19 @@ def test_pack_hand_computed():
     assert list(oracle.pack([7] * 13, 3)) == [0xFF, 0xFF, 0xFF, 0x3F, 0xFF, 0x01, 0x00, 0x00]
 
 
-@pytest.mark.parametrize("nbits", [2, 3, 4, 8])
+def test_pack_hand_computed_other_widths():
+    # 1 bit: eight codes per byte, the lowest index in the lowest bit.
+    # 1 + 0*2 + 1*4 + 1*8 + 0 + 0 + 0 + 1*128 = 141 = 0x8D; a ninth code starts the next byte
+    assert list(oracle.pack([1, 0, 1, 1, 0, 0, 0, 1, 1], 1)) == [0x8D, 0x01]
+    assert oracle.packed_bytes(64, 1) == 8 and oracle.packed_bytes(65, 1) == 9
+    # 5 and 6 bit [HQQ 算法解读, "为什么一定要分组"]: one code per byte, unpacked; 7 and 8 bit alike
+    for nbits in (5, 6, 7, 8):
+        top = (1 << nbits) - 1
+        assert list(oracle.pack([top, 0, 17], nbits)) == [top, 0, 17]
+        assert oracle.packed_bytes(64, nbits) == 64
+
+
+@pytest.mark.parametrize("nbits", [1, 2, 3, 4, 5, 6, 7, 8])
 @pytest.mark.parametrize("n", [1, 9, 10, 11, 64, 1001])
 def test_pack_roundtrip(nbits, n):
     rng = np.random.default_rng(n * 10 + nbits)
@@ -195,7 +207,7 @@ def test_group_error_is_mae_sum():
 
 
 # ------------------------------------------------------------------ the loop-free special case
-@pytest.mark.parametrize("nbits,g", [(4, 64), (3, 64), (2, 16)])
+@pytest.mark.parametrize("nbits,g", [(4, 64), (3, 64), (2, 16), (1, 32), (5, 64), (6, 64), (8, 128)])
 def test_iters0_is_minmax_rtn(nbits, g):
     # With no proximal iteration the method is asymmetric min-max RTN (k4i.top, sections
     # "线性量化：scale、zero point 与舍入" and "RTN：round-to-nearest 是基线").

@@ -1,8 +1,8 @@
 """Builds the CUDA library libhqq_b200.so in-tree with nvcc for sm_100a.
 
-The library is four translation units (the C ABI, the stream engine, the tile engine, and
-dequantize + the fused forward product), compiled in parallel and linked into one shared
-object.
+The library is five translation units (the C ABI, the stream engine, the tile engine in two
+parts, and dequantize + the fused forward product), compiled in parallel and linked into one
+shared object.
 """
 from __future__ import annotations
 
@@ -14,9 +14,10 @@ import subprocess
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-UNITS = ["hqq_abi.cu", "hqq_stream.cu", "hqq_tile.cu", "hqq_dequant.cu"]
+UNITS = ["hqq_abi.cu", "hqq_stream.cu", "hqq_tile_a.cu", "hqq_tile_b.cu", "hqq_dequant.cu"]
 SRCS = [os.path.join(CSRC, u) for u in UNITS]
-HDRS = [os.path.join(ROOT, "include", "hqq_b200.h"), os.path.join(CSRC, "hqq_common.cuh")]
+HDRS = [os.path.join(ROOT, "include", "hqq_b200.h"), os.path.join(CSRC, "hqq_common.cuh"),
+        os.path.join(CSRC, "hqq_tile.cuh")]
 LIB = os.path.join(HERE, "libhqq_b200.so")
 OBJ_DIR = os.path.join(HERE, "_build")
 

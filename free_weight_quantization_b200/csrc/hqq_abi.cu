@@ -22,12 +22,13 @@ int64_t gcd64(int64_t a, int64_t b) {
     return a;
 }
 
-int cpw_of(int nbits) { return nbits == 4 ? 8 : nbits == 2 ? 16 : 10; }
+// codes per 32-bit word of the packed layout (the Pack<NB> of the kernels)
+int cpw_of(int nbits) { return nbits == 3 ? 10 : nbits == 1 ? 32 : nbits == 2 ? 16 : nbits == 4 ? 8 : 4; }
 
 int make_plan(int64_t rows, int64_t cols, int nbits, int64_t group_size, int axis, int iters,
               Plan *pl) {
     if (rows <= 0 || cols <= 0 || group_size <= 0) return HQQ_ERR_ARG;
-    if (nbits != 2 && nbits != 3 && nbits != 4) return HQQ_ERR_ARG;
+    if (nbits < 1 || nbits > 8) return HQQ_ERR_ARG;
     if (axis != 0 && axis != 1) return HQQ_ERR_ARG;
     if (rows > (int64_t(1) << 40) / cols) return HQQ_ERR_UNSUPPORTED;
     const int64_t N = rows * cols;
@@ -45,12 +46,14 @@ int make_plan(int64_t rows, int64_t cols, int nbits, int64_t group_size, int axi
     pl->stride = P + (P >= 64 ? 8 : 0);  // halves per tile row (the padding staggers banks)
     const int target = 40960;            // halves of W per tile
     const int cap = std::max(1, target / pl->stride);
-    const int unit = axis == 1 ? (int)(320 / gcd64(pl->g, 320))  // tiles of 320k elements: word
-                               : 80;                             // (8, 16, 10 codes) and 16-byte
-    pl->tile = unit * std::max(1, cap / unit);                   // aligned; 80 = lcm(8, 16, 10)
+    // tiles that start on a packed word: axis 1, tiles of 320k elements (a multiple of 4, 8, 10,
+    // 16 and 32 codes, and 16-byte aligned); axis 0, a multiple of 80 columns (lcm of 4, 8, 10,
+    // 16), or of 160 for 1-bit codes (32 per word)
+    const int unit = axis == 1 ? (int)(320 / gcd64(pl->g, 320)) : (nbits == 1 ? 160 : 80);
+    pl->tile = unit * std::max(1, cap / unit);
     // two CTAs per SM: keep the whole shared-memory layout within 110 KB
     while (pl->tile > unit &&
-           smem_layout(pl->tile, pl->stride, 1 << nbits, pl->L, iters).total > 110 * 1024)
+           smem_layout(pl->tile, pl->stride, nbits <= 4 ? 1 << nbits : 0, pl->L, iters).total > 110 * 1024)
         pl->tile -= unit;
     // spread the groups evenly over whole waves of resident CTAs (two per SM)
     {
@@ -65,7 +68,7 @@ int make_plan(int64_t rows, int64_t cols, int nbits, int64_t group_size, int axi
     pl->aligned = axis == 1 || (pl->G % cpw_of(nbits) == 0);
     // the stream engine: axis 1, 2- and 4-bit codes, groups of 16 .. 128 that are whole 32-bit
     // words of the output (its codes are stored straight from registers)
-    pl->stream = axis == 1 && nbits != 3 && P <= 128 && pl->g == P && (pl->g * nbits) % 32 == 0;
+    pl->stream = axis == 1 && (nbits == 2 || nbits == 4) && P <= 128 && pl->g == P && (pl->g * nbits) % 32 == 0;
     const int K = iters > 0 ? iters : 1;
     pl->ws_acc = (size_t)4 * K * sizeof(u64) + 64;  // per-round sums + control words (zeroed)
     pl->ws_fk = (size_t)((pl->G + 15) / 16 * 16);
@@ -97,9 +100,11 @@ extern "C" void hqq_default_opt(hqq_opt_t *opt) {
 extern "C" int64_t hqq_packed_bytes(int64_t n, int nbits) {
     if (n < 0) return -1;
     switch (nbits) {
-    case 4: return (n + 1) / 2;
+    case 1: return (n + 7) / 8;
     case 2: return (n + 3) / 4;
     case 3: return 4 * ((n + 9) / 10);
+    case 4: return (n + 1) / 2;
+    case 5: case 6: case 7: case 8: return n;
     default: return -1;
     }
 }
@@ -176,7 +181,7 @@ extern "C" int hqq_quantize(const void *W, int64_t rows, int64_t cols, int nbits
     if (pl.stream) {
         e = hqq_impl::launch_stream_engine(P, nbits, pl.g, st);
     } else {
-        const bool direct = axis == 1 && pl.g % 16 == 0;
+        const bool direct = axis == 1 && pl.g % 16 == 0 && (nbits == 2 || nbits == 4);
         e = hqq_impl::launch_tile_engine(P, nbits, pl.L, pl.g == pl.P, direct, pl.ntiles, st);
     }
     return e == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;

@@ -114,11 +114,23 @@ __device__ __forceinline__ float seg_sum(float v) {
     return v;
 }
 
+// the packed layout of b-bit codes [HQQ 算法解读, "为什么一定要分组"]: cpw codes per 32-bit word,
+// each in a slot of `slot` bits, the lowest index in the lowest bits.  4 bit two per byte, 2 bit
+// four per byte, 3 bit ten per word; 5- and 6-bit codes one per byte (unpacked), and so 7 and 8
+// bit; 1-bit codes eight per byte.
 template <int NB>
-struct Pack;  // codes per 32-bit output word
-template <> struct Pack<4> { static constexpr int cpw = 8; };
-template <> struct Pack<2> { static constexpr int cpw = 16; };
-template <> struct Pack<3> { static constexpr int cpw = 10; };
+struct Pack {
+    static_assert(NB >= 1 && NB <= 8, "1- to 8-bit codes");
+    static constexpr int slot = NB == 3 ? 3 : NB <= 4 ? NB : 8;
+    static constexpr int cpw = NB == 3 ? 10 : 32 / slot;
+};
+// the tile engine reads W_hat = (k - z)/s from a table of the 2^b code values up to 4 bits; wider
+// codes divide per element (a 32..256-entry table per group and round would cost more)
+template <int NB>
+struct TileTab {
+    static constexpr bool on = NB <= 4;
+    static constexpr int nq = on ? (1 << NB) : 0;
+};
 
 
 // workspace words after the per-round sums: CTAs finished, kept round, rounds measured,
@@ -403,9 +415,13 @@ __device__ __forceinline__ u64 warp_sum64(u64 v) {
 // ------------------------------------------------------------------------------------------
 namespace hqq_impl {
 
-// the tile engine (axis 0, 3-bit, group sizes that are not whole power-of-two rows)
+// the tile engine (axis 0, 3-bit and the 1-, 5- to 8-bit codes, group sizes that are not whole
+// power-of-two rows); one launcher per code width, in two translation units
 cudaError_t launch_tile_engine(const QParams &P, int nbits, int L, bool full, bool direct,
                                int64_t ntiles, cudaStream_t st);
+template <int NB>
+cudaError_t launch_tile_nb(const QParams &P, int L, bool full, bool direct, int64_t ntiles,
+                           cudaStream_t st);
 // the stream engine (axis 1, 2- or 4-bit codes, group size 16, 32, 64 or 128)
 cudaError_t launch_stream_engine(const QParams &P, int nbits, int group_size, cudaStream_t st);
 cudaError_t launch_dequantize(int nbits, const uint8_t *pk, const __half *sc, const __half *ze,

@@ -68,7 +68,7 @@ __global__ void __launch_bounds__(kDqThreads) hqq_dequant_kernel(
 #pragma unroll
             for (int c = 0; c < CPW; ++c) {
                 const bool first = c < cb[u];
-                const float qf = __fsub_rn(__int_as_float(0x4B000000 | (int)((wd[u] >> (NB * c)) & MASK)), 8388608.0f);
+                const float qf = __fsub_rn(__int_as_float(0x4B000000 | (int)((wd[u] >> (Pack<NB>::slot * c)) & MASK)), 8388608.0f);
                 v[c] = __fmul_rn(__fsub_rn(qf, first ? z0[u] : z1[u]), first ? d0[u] : d1[u]);
             }
         } else if (MODE == 0) {
@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(kDqThreads) hqq_dequant_kernel(
             const float zf = __half2float(zero[k]), df = __half2float(scale[k]);
 #pragma unroll
             for (int c = 0; c < CPW; ++c) {
-                const float qf = __fsub_rn(__int_as_float(0x4B000000 | (int)((wd[u] >> (NB * c)) & MASK)), 8388608.0f);
+                const float qf = __fsub_rn(__int_as_float(0x4B000000 | (int)((wd[u] >> (Pack<NB>::slot * c)) & MASK)), 8388608.0f);
                 v[c] = __fmul_rn(__fsub_rn(qf, zf), df);
             }
         } else if (MODE == 2 && vec_meta) {
@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(kDqThreads) hqq_dequant_kernel(
                 const __half *dh = reinterpret_cast<const __half *>(&dv);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    const float qf = __fsub_rn(__int_as_float(0x4B000000 | (int)((wd[u] >> (NB * (c8 + c))) & MASK)), 8388608.0f);
+                    const float qf = __fsub_rn(__int_as_float(0x4B000000 | (int)((wd[u] >> (Pack<NB>::slot * (c8 + c))) & MASK)), 8388608.0f);
                     v[c8 + c] = __fmul_rn(__fsub_rn(qf, __half2float(zh[c])), __half2float(dh[c]));
                 }
             }
@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(kDqThreads) hqq_dequant_kernel(
             float zf = __half2float(zero[k]), df = __half2float(scale[k]);
 #pragma unroll
             for (int c = 0; c < CPW; ++c) {
-                const float qf = __fsub_rn(__int_as_float(0x4B000000 | (int)((wd[u] >> (NB * c)) & MASK)), 8388608.0f);
+                const float qf = __fsub_rn(__int_as_float(0x4B000000 | (int)((wd[u] >> (Pack<NB>::slot * c)) & MASK)), 8388608.0f);
                 v[c] = __fmul_rn(__fsub_rn(qf, zf), df);
                 if (c + 1 < CPW && n0 + c + 1 < N) {  // move to the group of the next element
                     if (MODE == 1) {
@@ -297,9 +297,9 @@ __global__ void __launch_bounds__(256) hqq_gemv_any_kernel(const uint8_t *__rest
         if (NB == 3) {
             const uint32_t wv = __ldg(reinterpret_cast<const uint32_t *>(packed) + n / 10);
             q = (wv >> (3 * (int)(n % 10))) & MASK;
-        } else {
-            const int per = 8 / NB;
-            q = ((uint32_t)__ldg(packed + n / per) >> (NB * (int)(n % per))) & MASK;
+        } else {  // slots of 1, 2, 4 or 8 bits inside bytes
+            constexpr int per = 8 / Pack<NB>::slot;
+            q = ((uint32_t)__ldg(packed + n / per) >> (Pack<NB>::slot * (int)(n % per))) & MASK;
         }
         const int64_t k = axis == 1 ? n / g : n % G;
         const float v = __fmul_rn(__fsub_rn((float)q, __half2float(__ldg(zero + k))), __half2float(__ldg(scale + k)));
@@ -317,13 +317,15 @@ cudaError_t launch_gemv_nb(const uint8_t *pk, const __half *sc, const __half *ze
     constexpr int CPW = Pack<NB>::cpw;
     const unsigned blocks = (unsigned)((rows + 7) / 8);
     const int64_t wpr = cols / CPW;
-    if (NB != 3 && axis == 1 && cols % CPW == 0 && g % CPW == 0 && ((uintptr_t)x & 15) == 0 &&
-        wpr < ((int64_t)1 << 30)) {
-        const int wpg = (int)(g / CPW);
-        int shift = -1;
-        if ((wpg & (wpg - 1)) == 0) { shift = 0; while ((1 << shift) < wpg) ++shift; }
-        return launch_pdl(hqq_gemv_kernel<NB>, blocks, 256, 0, st, (const uint32_t *)pk, sc, ze,
-                          rows, (int)wpr, (int)(cols / g), shift, wpg, x, y);
+    if constexpr (NB == 2 || NB == 4) {  // the fast path: 2- and 4-bit axis-1 layouts
+        if (axis == 1 && cols % CPW == 0 && g % CPW == 0 && ((uintptr_t)x & 15) == 0 &&
+            wpr < ((int64_t)1 << 30)) {
+            const int wpg = (int)(g / CPW);
+            int shift = -1;
+            if ((wpg & (wpg - 1)) == 0) { shift = 0; while ((1 << shift) < wpg) ++shift; }
+            return launch_pdl(hqq_gemv_kernel<NB>, blocks, 256, 0, st, (const uint32_t *)pk, sc, ze,
+                              rows, (int)wpr, (int)(cols / g), shift, wpg, x, y);
+        }
     }
     return launch_pdl(hqq_gemv_any_kernel<NB>, blocks, 256, 0, st, pk, sc, ze, rows, cols, g, G,
                       axis, x, y);
@@ -337,9 +339,14 @@ cudaError_t launch_dequantize(int nbits, const uint8_t *pk, const __half *sc, co
                               int64_t N, int g, int64_t G, int axis, int64_t pb, __half *out,
                               cudaStream_t st) {
     switch (nbits) {
-    case 4: return launch_dequant<4>(pk, sc, ze, N, g, G, axis, pb, out, st);
+    case 1: return launch_dequant<1>(pk, sc, ze, N, g, G, axis, pb, out, st);
+    case 2: return launch_dequant<2>(pk, sc, ze, N, g, G, axis, pb, out, st);
     case 3: return launch_dequant<3>(pk, sc, ze, N, g, G, axis, pb, out, st);
-    default: return launch_dequant<2>(pk, sc, ze, N, g, G, axis, pb, out, st);
+    case 4: return launch_dequant<4>(pk, sc, ze, N, g, G, axis, pb, out, st);
+    case 5: return launch_dequant<5>(pk, sc, ze, N, g, G, axis, pb, out, st);
+    case 6: return launch_dequant<6>(pk, sc, ze, N, g, G, axis, pb, out, st);
+    case 7: return launch_dequant<7>(pk, sc, ze, N, g, G, axis, pb, out, st);
+    default: return launch_dequant<8>(pk, sc, ze, N, g, G, axis, pb, out, st);
     }
 }
 
@@ -347,9 +354,14 @@ cudaError_t launch_gemv(int nbits, const uint8_t *pk, const __half *sc, const __
                         int64_t rows, int64_t cols, int64_t g, int64_t G, int axis,
                         const __half *x, float *y, cudaStream_t st) {
     switch (nbits) {
-    case 4: return launch_gemv_nb<4>(pk, sc, ze, rows, cols, g, G, axis, x, y, st);
+    case 1: return launch_gemv_nb<1>(pk, sc, ze, rows, cols, g, G, axis, x, y, st);
+    case 2: return launch_gemv_nb<2>(pk, sc, ze, rows, cols, g, G, axis, x, y, st);
     case 3: return launch_gemv_nb<3>(pk, sc, ze, rows, cols, g, G, axis, x, y, st);
-    default: return launch_gemv_nb<2>(pk, sc, ze, rows, cols, g, G, axis, x, y, st);
+    case 4: return launch_gemv_nb<4>(pk, sc, ze, rows, cols, g, G, axis, x, y, st);
+    case 5: return launch_gemv_nb<5>(pk, sc, ze, rows, cols, g, G, axis, x, y, st);
+    case 6: return launch_gemv_nb<6>(pk, sc, ze, rows, cols, g, G, axis, x, y, st);
+    case 7: return launch_gemv_nb<7>(pk, sc, ze, rows, cols, g, G, axis, x, y, st);
+    default: return launch_gemv_nb<8>(pk, sc, ze, rows, cols, g, G, axis, x, y, st);
     }
 }
 

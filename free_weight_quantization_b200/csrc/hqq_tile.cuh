@@ -1,4 +1,4 @@
-// hqq_tile.cu -- the tile engine of the B200 HQQ quantizer: axis 0 (groups strided along the
+// hqq_tile.cuh -- the tile engine of the B200 HQQ quantizer: axis 0 (groups strided along the
 // output dimension), 3-bit codes, and group sizes that are not whole power-of-two rows.
 //
 // One CTA of 256 threads per tile of groups staged in shared memory [HQQ 算法解读, "`axis` 不是
@@ -6,6 +6,8 @@
 // round after round until its zero stops moving or `iters` rounds are done; exact per-round
 // error counters, the stop rule in the last CTA to finish, and a fixup kernel that replays the
 // groups whose own last round lies past the kept one.
+#pragma once
+
 #include <algorithm>
 
 #include "hqq_common.cuh"
@@ -151,7 +153,7 @@ struct Codes {
 // the code table, |W - W_hat| and q - W*s (the zero-update term with e = 0); the codes are
 // kept.  CLIP = false only when every t of the warp's groups rounds inside [0, 2^b - 1].
 template <int NB, int NSEG, bool CLIP, bool FULL, bool DIRECT>
-__device__ __forceinline__ void round_elems(const float (&w)[kE], const float (&ws)[kE], float z,
+__device__ __forceinline__ void round_elems(const float (&w)[kE], const float (&ws)[kE], float s, float z,
                                             uint32_t tab_adj, int nvalid, float (&absr)[kE],
                                             float (&term)[kE], Codes<NB, DIRECT> &codes) {
     constexpr int NQ = 1 << NB;
@@ -167,7 +169,10 @@ __device__ __forceinline__ void round_elems(const float (&w)[kE], const float (&
         // tab_adj + (bits << kShift) (mod 2^32), tab_adj having absorbed the constant part
         const uint32_t bits = __float_as_uint(u);
         float what;
-        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(what) : "r"(tab_adj + (bits << kShift)));
+        if constexpr (TileTab<NB>::on)
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(what) : "r"(tab_adj + (bits << kShift)));
+        else
+            what = __fdiv_rn(__fsub_rn(qf, z), s);  // (q - z)/s, the IEEE division itself
         codes.put(m, bits);
         const float ar = fabsf(__fsub_rn(w[m], what));
         const float tm = __fsub_rn(qf, ws[m]);        // q - (W - 0)*s
@@ -296,16 +301,18 @@ __device__ void run_groups(const QParams &P, __half *wh, const float *s_t, float
             const bool noclip = __all_sync(kFull, inside);
             // reconstructions W_hat = (k - z)/s for every code k: the IEEE division of the
             // method, done once per code value instead of once per element
-            __syncwarp();
+            if constexpr (TileTab<NB>::on) {
+                __syncwarp();
 #pragma unroll
-            for (int kk = 0; kk < (NQ + L - 1) / L; ++kk) {
-                const int k = l + kk * L;
-                if (k < NQ) tab[k * NSEG + sg] = __fdiv_rn(__fsub_rn(lf + (float)(kk * L), z), s);
+                for (int kk = 0; kk < (NQ + L - 1) / L; ++kk) {
+                    const int k = l + kk * L;
+                    if (k < NQ) tab[k * NSEG + sg] = __fdiv_rn(__fsub_rn(lf + (float)(kk * L), z), s);
+                }
+                __syncwarp();
             }
-            __syncwarp();
             float absr[kE], term[kE];
-            if (noclip) round_elems<NB, NSEG, false, FULL, DIRECT>(w, ws, z, tab_adj, nvalid, absr, term, codes);
-            else round_elems<NB, NSEG, true, FULL, DIRECT>(w, ws, z, tab_adj, nvalid, absr, term, codes);
+            if (noclip) round_elems<NB, NSEG, false, FULL, DIRECT>(w, ws, s, z, tab_adj, nvalid, absr, term, codes);
+            else round_elems<NB, NSEG, true, FULL, DIRECT>(w, ws, s, z, tab_adj, nvalid, absr, term, codes);
             const float esum_l = tree16(absr);
             // the lane's largest residual is at most its partial sum; only when that bound
             // fails is the maximum taken
@@ -327,7 +334,8 @@ __device__ void run_groups(const QParams &P, __half *wh, const float *s_t, float
                     t = fminf(fmaxf(t, 0.0f), kQmax);
                     const float u = __fadd_rn(t, kMagic);
                     const float qf = __fsub_rn(u, kMagic);
-                    const float what = tab[(__float_as_int(u) & (NQ - 1)) * NSEG + sg];
+                    const float what = TileTab<NB>::on ? tab[(__float_as_int(u) & (NQ - 1)) * NSEG + sg]
+                                                       : __fdiv_rn(__fsub_rn(qf, z), s);
                     const float rr = __fsub_rn(w[m], what);
                     const float e = (slow && m < nvalid) ? shrink_lp(rr, beta, P.p) : 0.0f;
                     term[m] = (m < nvalid) ? __fsub_rn(qf, __fmul_rn(__fsub_rn(w[m], e), s)) : 0.0f;
@@ -440,7 +448,7 @@ __device__ void write_tile(const QParams &P, const __half *wh, const float *s_t,
 #pragma unroll
             for (int k = 0; k < CPW; ++k) {
                 if (e0 + k < ne) {
-                    word |= (uint32_t)cb[grp * rowb + j] << (NB * k);
+                    word |= (uint32_t)cb[grp * rowb + j] << (Pack<NB>::slot * k);
                     if (++j == g) { j = 0; ++grp; }
                 }
             }
@@ -456,7 +464,7 @@ __device__ void write_tile(const QParams &P, const __half *wh, const float *s_t,
 #pragma unroll
             for (int k = 0; k < CPW; ++k) {
                 const int col = wr * CPW + k;
-                if (col < tg) word |= (uint32_t)cb[col * rowb + j] << (NB * k);
+                if (col < tg) word |= (uint32_t)cb[col * rowb + j] << (Pack<NB>::slot * k);
             }
             store_word((j * P.G + t0) / CPW + wr, word);
         }
@@ -472,14 +480,14 @@ struct Smem {
     unsigned *acc;    // all warps' counters
     unsigned *acc_w;  // this warp's counters
     __device__ Smem(unsigned char *base, const QParams &P) {
-        const SmemLayout lay = smem_layout(P.tile, P.stride, 1 << NB, L, P.K);
+        const SmemLayout lay = smem_layout(P.tile, P.stride, TileTab<NB>::nq, L, P.K);
         wh = reinterpret_cast<__half *>(base + lay.wh);
         s_t = reinterpret_cast<float *>(base + lay.s_t);
         z_t = reinterpret_cast<float *>(base + lay.z_t);
         lo_t = reinterpret_cast<float *>(base + lay.lo_t);
         hi_t = reinterpret_cast<float *>(base + lay.hi_t);
         f_t = base + lay.f_t;
-        tab = reinterpret_cast<float *>(base + lay.tab) + (threadIdx.x >> 5) * (1 << NB) * (32 / L);
+        tab = reinterpret_cast<float *>(base + lay.tab) + (threadIdx.x >> 5) * TileTab<NB>::nq * (32 / L);
         acc = reinterpret_cast<unsigned *>(base + lay.acc);
         acc_w = acc + (threadIdx.x >> 5) * 8 * (P.K > 0 ? P.K : 1);
         thr = reinterpret_cast<float *>(base + lay.thr);
@@ -596,7 +604,7 @@ __global__ void pack_codes_kernel(const uint8_t *codes, int64_t N, uint8_t *pack
         uint32_t word = 0;
         for (int c = 0; c < CPW; ++c) {
             const int64_t n = wi * CPW + c;
-            if (n < N) word |= (uint32_t)codes[n] << (NB * c);
+            if (n < N) word |= (uint32_t)codes[n] << (Pack<NB>::slot * c);
         }
         const int64_t off = wi * 4;
         if (off + 4 <= packed_bytes) {
@@ -611,7 +619,7 @@ __global__ void pack_codes_kernel(const uint8_t *codes, int64_t N, uint8_t *pack
 // ---- host side
 template <int NB, int L, bool FULL, bool DIRECT>
 cudaError_t launch_quant(const QParams &P, int64_t ntiles, cudaStream_t st) {
-    const SmemLayout lay = smem_layout(P.tile, P.stride, 1 << NB, L, P.K);
+    const SmemLayout lay = smem_layout(P.tile, P.stride, TileTab<NB>::nq, L, P.K);
     cudaError_t e = cudaFuncSetAttribute(hqq_search_kernel<NB, L, FULL, DIRECT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total);
     if (e != cudaSuccess) return e;
@@ -652,9 +660,10 @@ cudaError_t launch_quant_l(const QParams &P, int L, int64_t ntiles, cudaStream_t
 template <int NB>
 cudaError_t launch_quant_nb(const QParams &P, int L, bool full, bool direct, int64_t ntiles,
                             cudaStream_t st) {
-    if (NB != 3 && direct && L == 16)
-        return full ? launch_quant<NB, 16, true, NB != 3>(P, ntiles, st)
-                    : launch_quant<NB, 16, false, NB != 3>(P, ntiles, st);
+    constexpr bool kDirect = NB == 2 || NB == 4;
+    if (kDirect && direct && L == 16)
+        return full ? launch_quant<NB, 16, true, kDirect>(P, ntiles, st)
+                    : launch_quant<NB, 16, false, kDirect>(P, ntiles, st);
     return full ? launch_quant_l<NB, true, false>(P, L, ntiles, st)
                 : launch_quant_l<NB, false, false>(P, L, ntiles, st);
 }
@@ -664,13 +673,10 @@ cudaError_t launch_quant_nb(const QParams &P, int L, bool full, bool direct, int
 
 namespace hqq_impl {
 
-cudaError_t launch_tile_engine(const QParams &P, int nbits, int L, bool full, bool direct,
-                               int64_t ntiles, cudaStream_t st) {
-    switch (nbits) {
-    case 4: return launch_quant_nb<4>(P, L, full, direct, ntiles, st);
-    case 3: return launch_quant_nb<3>(P, L, full, false, ntiles, st);
-    default: return launch_quant_nb<2>(P, L, full, direct, ntiles, st);
-    }
+template <int NB>
+cudaError_t launch_tile_nb(const QParams &P, int L, bool full, bool direct, int64_t ntiles,
+                           cudaStream_t st) {
+    return launch_quant_nb<NB>(P, L, full, direct, ntiles, st);
 }
 
 }  // namespace hqq_impl

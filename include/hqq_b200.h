@@ -18,8 +18,10 @@
  *     the [g, G] row-major view (W.reshape([g, -1])), i.e. group k = elements j*G + k;
  *   - packed codes are in flat row-major element order for both axes, lowest index in the
  *     lowest bits [HQQ 算法解读, "为什么一定要分组"]: 4 bit = two codes per byte, 2 bit = four
- *     codes per byte, 3 bit = ten codes per little-endian 32-bit word (bits 30-31 zero); the
- *     tail of the last byte or word is zero;
+ *     codes per byte, 3 bit = ten codes per little-endian 32-bit word (bits 30-31 zero),
+ *     5 and 6 bit = one code per byte (unpacked); this library stores 7- and 8-bit codes one
+ *     per byte as well and packs 1-bit codes eight per byte (the pages name 1 bit without a
+ *     layout); the tail of the last byte or word is zero;
  *   - metadata [HQQ 算法解读, "量化公式：把尺子写出来"]: scale[G] = fp16(1/s) (the page's
  *     Delta) and zero[G] = fp16(z), in group order.
  *   - W should hold finite values: a group with a NaN or an infinity gets unspecified codes and
@@ -69,8 +71,9 @@ typedef struct hqq_opt {
 /* Fills *opt with the page's defaults: 20, 0.7, 10, 1.01, 1e-4, 2e4. */
 void hqq_default_opt(hqq_opt_t *opt);
 
-/* Exact size in bytes of the packed codes of n weights: n/2, n/4 or 4*ceil(n/10), rounded up
- * [HQQ 算法解读, "为什么一定要分组"].  Returns -1 for nbits outside {2, 3, 4} or n < 0. */
+/* Exact size in bytes of the packed codes of n weights [HQQ 算法解读, "为什么一定要分组"]:
+ * n/8 (1 bit), n/4 (2 bit), 4*ceil(n/10) (3 bit), n/2 (4 bit), rounded up, or n (5 to 8 bit).
+ * Returns -1 for nbits outside 1..8 or n < 0. */
 int64_t hqq_packed_bytes(int64_t n, int nbits);
 
 /* Device workspace, in bytes, that hqq_quantize needs for these arguments (0 if invalid). */
@@ -88,7 +91,10 @@ size_t hqq_quantize_workspace_bytes(int64_t rows, int64_t cols, int nbits, int64
  *
  * Arguments
  *   W            [rows*cols] fp16, 16-byte aligned
- *   nbits        2, 3 or 4;  group_size 1..256 dividing rows*cols;  axis 0 or 1
+ *   nbits        1 to 8;  group_size 1..256 dividing rows*cols;  axis 0 or 1.  2- and 4-bit
+ *                axis-1 layouts with a power-of-two group of 16..128 run the one-group-per-lane
+ *                engine; every other layout the tile engine, which for 5 to 8 bits computes
+ *                W_hat by one IEEE division per element instead of a table of the 2^b values
  *   opt          options (host pointer); NULL = hqq_default_opt()
  *   packed       [hqq_packed_bytes(N, nbits)] bytes, 16-byte aligned (output)
  *   scale, zero  [G] fp16 each, 2-byte aligned (outputs): fp16(1/s) and fp16(z)

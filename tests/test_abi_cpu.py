@@ -42,14 +42,15 @@ def test_default_opt_is_the_pages_defaults(L):
     assert abs(o.eps_tiny - 1e-4) < 1e-9 and o.scale_max == 2e4
 
 
-@pytest.mark.parametrize("nbits", [2, 3, 4])
+@pytest.mark.parametrize("nbits", [1, 2, 3, 4, 5, 6, 7, 8])
 @pytest.mark.parametrize("n", [0, 1, 7, 10, 64, 4096 * 4096, 4096 * 11008 + 3])
 def test_packed_bytes_match_oracle(L, nbits, n):
     assert hqq.hqq_packed_bytes(n, nbits) == oracle.packed_bytes(n, nbits)
 
 
 def test_packed_bytes_rejects(L):
-    assert hqq.hqq_packed_bytes(10, 5) == -1
+    assert hqq.hqq_packed_bytes(10, 9) == -1
+    assert hqq.hqq_packed_bytes(10, 0) == -1
     assert hqq.hqq_packed_bytes(-1, 4) == -1
 
 
@@ -60,7 +61,9 @@ def test_workspace_bytes(L):
     G = 4096 * 4096 // 64
     assert G <= ws(4096, 4096, 4, 64, 1, 20) < G + 65536
     assert ws(10, 10, 4, 3, 1, 20) == 0        # 100 % 3 != 0
-    assert ws(16, 16, 5, 16, 1, 20) == 0       # 5 bits
+    assert ws(16, 16, 9, 16, 1, 20) == 0       # 9 bits
+    assert ws(16, 16, 0, 16, 1, 20) == 0       # 0 bits
+    assert ws(16, 16, 5, 16, 1, 20) > 0        # 5 bits: the tile engine
     assert ws(16, 16, 4, 16, 2, 20) == 0       # axis 2
     assert ws(16, 1024, 4, 512, 1, 20) == 0    # group beyond the library limit
     assert ws(16, 16, 4, 16, 1, 65) == 0       # iters beyond the library limit
@@ -80,8 +83,8 @@ def q(L, W=FAKE, rows=64, cols=64, nbits=4, g=64, axis=1, opt=None, packed=FAKE,
 
 
 def test_quantize_rejects_on_host(L):
-    assert q(L, nbits=5) == 1
-    assert q(L, nbits=1) == 1
+    assert q(L, nbits=9) == 1
+    assert q(L, nbits=0) == 1
     assert q(L, axis=3) == 1
     assert q(L, g=0) == 1
     assert q(L, rows=0) == 1
@@ -108,7 +111,7 @@ def test_quantize_rejects_on_host(L):
 def test_dequantize_rejects_on_host(L):
     P = ctypes.c_void_p
     d = L.hqq_dequantize
-    assert d(P(FAKE), P(FAKE), P(FAKE), 64, 64, 5, 64, 1, P(FAKE), None) == 1
+    assert d(P(FAKE), P(FAKE), P(FAKE), 64, 64, 9, 64, 1, P(FAKE), None) == 1
     assert d(P(FAKE), P(FAKE), P(FAKE), 64, 64, 4, 63, 1, P(FAKE), None) == 1
     assert d(None, P(FAKE), P(FAKE), 64, 64, 4, 64, 1, P(FAKE), None) == 1
     assert d(P(FAKE + 4), P(FAKE), P(FAKE), 64, 64, 4, 64, 1, P(FAKE), None) == 2
@@ -131,7 +134,8 @@ def test_gemv_rejects_on_host(L):
         a = args(**k)
         return gv(P(a["pk"]), P(a["sc"]), P(a["ze"]), a["rows"], a["cols"], a["nb"], a["g"],
                   a["ax"], P(a["x"]) if a["x"] else None, P(a["y"]) if a["y"] else None, None)
-    assert call(nb=5) == 1
+    assert call(nb=9) == 1
+    assert call(nb=0) == 1
     assert call(g=48) == 1                 # 4096 % 48 != 0
     assert call(ax=2) == 1
     assert call(x=0) == 1

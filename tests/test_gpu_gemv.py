@@ -44,7 +44,10 @@ LAYOUTS = [(4, 64, 1, 96, 512), (2, 16, 1, 64, 256), (4, 128, 1, 33, 1024), (2, 
            (3, 64, 1, 40, 640), (3, 10, 1, 21, 130), (4, 64, 0, 64, 192), (2, 16, 0, 48, 80),
            (4, 3, 1, 30, 21), (4, 24, 1, 12, 96),
            # one word per row, a ragged last CTA of rows, the largest group, one row
-           (4, 8, 1, 7, 8), (2, 16, 1, 1, 16), (4, 256, 1, 9, 4096), (2, 256, 1, 3, 8192)]
+           (4, 8, 1, 7, 8), (2, 16, 1, 1, 16), (4, 256, 1, 9, 4096), (2, 256, 1, 3, 8192),
+           # the other code widths (generic path): 1 bit eight per byte, 5 to 8 bit one per byte
+           (1, 64, 1, 16, 512), (1, 32, 0, 24, 100), (5, 32, 1, 20, 256), (6, 64, 0, 64, 96),
+           (7, 16, 1, 8, 64), (8, 64, 1, 33, 192)]
 
 
 @pytest.mark.parametrize("nbits,g,axis,rows,cols", LAYOUTS, ids=lambda v: str(v))

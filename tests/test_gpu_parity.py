@@ -108,6 +108,16 @@ EDGE = [
     (64, 256, 2, 16, 1, 20, "pos"),
     (64, 256, 3, 64, 1, 20, "neg"),
     (64, 256, 4, 64, 0, 20, "pos"),
+    # the other code widths: 1 bit (eight per byte), 5 to 8 bit (one per byte)
+    (64, 256, 1, 64, 1, 20, "t"),
+    (33, 96, 1, 32, 0, 20, "t"),           # axis 0, G = 99: byte staging + pack kernel
+    (64, 256, 5, 64, 1, 20, "t"),
+    (40, 160, 6, 32, 1, 20, "n"),
+    (64, 256, 7, 128, 0, 20, "t"),
+    (64, 256, 8, 64, 1, 20, "t"),
+    (48, 100, 8, 25, 1, 20, "wide"),       # odd group, shrink active
+    (64, 256, 6, 64, 1, 20, "bimodal"),    # early global stop with 6-bit codes
+    (64, 256, 8, 64, 1, 0, "t"),           # no rounds: min-max RTN at 8 bit
 ]
 
 
@@ -140,7 +150,7 @@ def test_full_size_config(case, pool):
     print(case.name, ref["iters_run"], stats)
 
 
-@pytest.mark.parametrize("nbits", [2, 3, 4])
+@pytest.mark.parametrize("nbits", [1, 2, 3, 4, 5, 6, 7, 8])
 @pytest.mark.parametrize("shape,g,axis", [((64, 64), 64, 1), ((37, 129), 3, 1), ((100, 7), 10, 1),
                                           ((256, 64), 128, 0), ((30, 32), 16, 0),
                                           ((41, 40), 8, 0)])

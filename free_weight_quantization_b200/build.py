@@ -1,8 +1,8 @@
 """Builds the CUDA library libhqq_b200.so in-tree with nvcc for sm_100a.
 
-The library is five translation units (the C ABI, the stream engine, the tile engine in two
-parts, and dequantize + the fused forward product), compiled in parallel and linked into one
-shared object.
+The library is six translation units (the C ABI, the stream engine, the tile engine in two
+parts, dequantize + the one-vector forward product, and the tensor-core product of a batch),
+compiled in parallel and linked into one shared object.
 """
 from __future__ import annotations
 
@@ -14,7 +14,8 @@ import subprocess
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-UNITS = ["hqq_abi.cu", "hqq_stream.cu", "hqq_tile_a.cu", "hqq_tile_b.cu", "hqq_dequant.cu"]
+UNITS = ["hqq_abi.cu", "hqq_stream.cu", "hqq_tile_a.cu", "hqq_tile_b.cu", "hqq_dequant.cu",
+         "hqq_gemm.cu"]
 SRCS = [os.path.join(CSRC, u) for u in UNITS]
 HDRS = [os.path.join(ROOT, "include", "hqq_b200.h"), os.path.join(CSRC, "hqq_common.cuh"),
         os.path.join(CSRC, "hqq_tile.cuh")]

@@ -223,6 +223,33 @@ extern "C" int hqq_gemv(const void *packed, const void *scale, const void *zero,
     return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
 }
 
+extern "C" int hqq_gemm(const void *packed, const void *scale, const void *zero, int64_t rows,
+                        int64_t cols, int nbits, int64_t group_size, int axis, const void *X,
+                        int64_t batch, float *Y, void *stream) {
+    Plan pl;
+    int rc = make_plan(rows, cols, nbits, group_size, axis, 0, &pl);
+    if (rc != HQQ_OK) return rc;
+    if (batch < 0) return HQQ_ERR_ARG;
+    if (batch == 0) return HQQ_OK;
+    if (!packed || !scale || !zero || !X || !Y) return HQQ_ERR_ARG;
+    if (!aligned_to(packed, 16) || !aligned_to(scale, 2) || !aligned_to(zero, 2) ||
+        !aligned_to(X, 2) || !aligned_to(Y, 4))
+        return HQQ_ERR_ALIGN;
+    cudaStream_t st = (cudaStream_t)stream;
+    const uint8_t *pk = (const uint8_t *)packed;
+    const __half *sc = (const __half *)scale, *ze = (const __half *)zero, *xh = (const __half *)X;
+    cudaError_t e;
+    if (hqq_impl::gemm_tc_layout(nbits, rows, cols, pl.g, axis, X)) {
+        e = hqq_impl::launch_gemm_tc(nbits, pk, sc, ze, rows, cols, pl.g, xh, batch, Y, st);
+    } else {  // any other layout: the generic product, one batch entry at a time
+        e = cudaSuccess;
+        for (int64_t b = 0; b < batch && e == cudaSuccess; ++b)
+            e = hqq_impl::launch_gemv(nbits, pk, sc, ze, rows, cols, pl.g, pl.G, axis, xh + b * cols,
+                                      Y + b * rows, st);
+    }
+    return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
+}
+
 extern "C" const char *hqq_strerror(int code) {
     switch (code) {
     case HQQ_OK: return "ok";

@@ -427,6 +427,12 @@ cudaError_t launch_stream_engine(const QParams &P, int nbits, int group_size, cu
 cudaError_t launch_dequantize(int nbits, const uint8_t *pk, const __half *sc, const __half *ze,
                               int64_t N, int g, int64_t G, int axis, int64_t pb, __half *out,
                               cudaStream_t st);
+// the tensor-core product of a batch (axis 1, 2- or 4-bit codes, group size a multiple of 8,
+// cols a multiple of 64, X 16-byte aligned)
+bool gemm_tc_layout(int nbits, int64_t rows, int64_t cols, int64_t g, int axis, const void *X);
+cudaError_t launch_gemm_tc(int nbits, const uint8_t *pk, const __half *sc, const __half *ze,
+                           int64_t rows, int64_t cols, int64_t g, const __half *X, int64_t batch,
+                           float *Y, cudaStream_t st);
 cudaError_t launch_gemv(int nbits, const uint8_t *pk, const __half *sc, const __half *ze,
                         int64_t rows, int64_t cols, int64_t g, int64_t G, int axis,
                         const __half *x, float *y, cudaStream_t st);

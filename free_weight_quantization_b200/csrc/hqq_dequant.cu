@@ -318,7 +318,8 @@ cudaError_t launch_gemv_nb(const uint8_t *pk, const __half *sc, const __half *ze
     const unsigned blocks = (unsigned)((rows + 7) / 8);
     const int64_t wpr = cols / CPW;
     if constexpr (NB == 2 || NB == 4) {  // the fast path: 2- and 4-bit axis-1 layouts
-        if (axis == 1 && cols % CPW == 0 && g % CPW == 0 && ((uintptr_t)x & 15) == 0 &&
+        // groups must not cross rows (cols % g == 0): the kernel finds a word's group by row
+        if (axis == 1 && cols % CPW == 0 && g % CPW == 0 && cols % g == 0 && ((uintptr_t)x & 15) == 0 &&
             wpr < ((int64_t)1 << 30)) {
             const int wpg = (int)(g / CPW);
             int shift = -1;

@@ -45,6 +45,7 @@ SIGNATURES = {
     "hqq_quantize_noalloc": (_I32, [_P, _I64, _I64, _I32, _I64, _I32, ctypes.POINTER(HqqOpt), _P,
                                     _P, _P, _P, _P, _P, _P, _P, _P]),
     "hqq_gemv": (_I32, [_P, _P, _P, _I64, _I64, _I32, _I64, _I32, _P, _P, _P]),
+    "hqq_gemm": (_I32, [_P, _P, _P, _I64, _I64, _I32, _I64, _I32, _P, _I64, _P, _P]),
     "hqq_strerror": (ctypes.c_char_p, [_I32]),
 }
 
@@ -204,6 +205,22 @@ def hqq_gemv(q: Quantized, x: torch.Tensor, out: torch.Tensor | None = None,
     rc = lib().hqq_gemv(_ptr(q.packed), _ptr(q.scale), _ptr(q.zero), q.rows, q.cols, q.nbits,
                         q.group_size, q.axis, _ptr(x), _ptr(out), ctypes.c_void_p(st.cuda_stream))
     _check(rc, "hqq_gemv")
+    return out
+
+
+def hqq_gemm(q: Quantized, X: torch.Tensor, out: torch.Tensor | None = None,
+             stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """Y = X @ W_hat.T for a batch of inputs with dequantization fused in (see hqq_gemm in the
+    header): X is a contiguous fp16 CUDA matrix [batch, cols], Y binary32 [batch, rows]."""
+    if X.dtype != torch.float16 or not X.is_cuda or X.dim() != 2 or X.shape[1] != q.cols or not X.is_contiguous():
+        raise HqqError("X must be a contiguous fp16 CUDA matrix [batch, cols]")
+    batch = X.shape[0]
+    if out is None:
+        out = torch.empty(batch, q.rows, dtype=torch.float32, device=q.packed.device)
+    st = stream if stream is not None else torch.cuda.current_stream(q.packed.device)
+    rc = lib().hqq_gemm(_ptr(q.packed), _ptr(q.scale), _ptr(q.zero), q.rows, q.cols, q.nbits,
+                        q.group_size, q.axis, _ptr(X), batch, _ptr(out), ctypes.c_void_p(st.cuda_stream))
+    _check(rc, "hqq_gemm")
     return out
 
 

@@ -146,12 +146,36 @@ int hqq_dequantize(const void *packed, const void *scale, const void *zero, int6
  *   y       [rows] binary32, 4-byte aligned (output)
  *   stream  cudaStream_t, or NULL for the default stream
  * Every layout is accepted. The fast path (one warp per output row) needs axis 1, 2- or 4-bit
- * codes, and cols and group_size multiples of the codes per 32-bit word (8 at 4 bit, 16 at 2
- * bit). Other layouts read their codes one at a time.
+ * codes, cols and group_size multiples of the codes per 32-bit word (8 at 4 bit, 16 at 2 bit),
+ * and group_size dividing cols. Other layouts read their codes one at a time.
  * Returns HQQ_OK, HQQ_ERR_ARG (shape or null pointer), HQQ_ERR_ALIGN, or HQQ_ERR_CUDA.
  */
 int hqq_gemv(const void *packed, const void *scale, const void *zero, int64_t rows, int64_t cols,
              int nbits, int64_t group_size, int axis, const void *x, float *y, void *stream);
+
+/*
+ * hqq_gemm: the quantized layer's forward product for a batch of input vectors, with
+ * dequantization fused in [HQQ 算法解读, "从压缩文件到一次前向"; the `axis` table's row for low-batch
+ * inference throughput]:
+ *     Y[b, r] = sum_c W_hat[r, c] * X[b, c]        for b < batch
+ * W_hat[r, c] is exactly the fp16 value hqq_dequantize writes.  Each product of two fp16 values is
+ * exact in binary32 and the sums run in binary32 in an order of the library's choosing, so
+ * Y[b, r] is within cols * 2^-23 * sum_c |W_hat[r, c] * X[b, c]| of the exact sum.
+ *   packed, scale, zero  as written by hqq_quantize (packed 16-byte aligned, scale and zero
+ *                        2-byte aligned)
+ *   X       [batch, cols] fp16 row-major, 2-byte aligned
+ *   batch   >= 0 (0: nothing is launched)
+ *   Y       [batch, rows] binary32 row-major, 4-byte aligned (output)
+ *   stream  cudaStream_t, or NULL for the default stream
+ * Axis-1 layouts with 2- or 4-bit codes, group_size a multiple of 8 that divides cols, cols a
+ * multiple of 64 and a 16-byte aligned X run on the tensor cores (tcgen05.mma, fp16 operands, binary32 accumulators in
+ * tensor memory; up to 256 batch entries per launch).  Every other layout runs the one-vector
+ * product once per batch entry.
+ * Returns HQQ_OK, HQQ_ERR_ARG (shape, batch or null pointer), HQQ_ERR_ALIGN, or HQQ_ERR_CUDA.
+ */
+int hqq_gemm(const void *packed, const void *scale, const void *zero, int64_t rows, int64_t cols,
+             int nbits, int64_t group_size, int axis, const void *X, int64_t batch, float *Y,
+             void *stream);
 
 /*
  * hqq_quantize without a workspace argument.  The pages have no counterpart to this call: it

@@ -224,6 +224,17 @@ def gemv(packed, scale, zero, rows: int, cols: int, nbits: int, group_size: int,
     return y, mag
 
 
+def gemm(packed, scale, zero, rows: int, cols: int, nbits: int, group_size: int, axis: int,
+         X) -> tuple[np.ndarray, np.ndarray]:
+    """Y = X @ W_hat.T for a batch X [batch, cols] fp16: hqo_gemv for every row of X (the
+    product is defined row by row); returns Y and the per-element sum of |W_hat * x|, both
+    [batch, rows] binary64."""
+    X = np.ascontiguousarray(X, dtype=np.float16)
+    out = [gemv(packed, scale, zero, rows, cols, nbits, group_size, axis, x) for x in X]
+    return (np.stack([y for y, _ in out]) if out else np.zeros((0, rows))), \
+           (np.stack([m for _, m in out]) if out else np.zeros((0, rows)))
+
+
 def dequant(packed, scale, zero, rows: int, cols: int, nbits: int, group_size: int,
             axis: int = 1) -> np.ndarray:
     """Unpack + (q - z)*Delta -> fp16 [rows, cols]."""

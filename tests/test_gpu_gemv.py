@@ -47,7 +47,9 @@ LAYOUTS = [(4, 64, 1, 96, 512), (2, 16, 1, 64, 256), (4, 128, 1, 33, 1024), (2, 
            (4, 8, 1, 7, 8), (2, 16, 1, 1, 16), (4, 256, 1, 9, 4096), (2, 256, 1, 3, 8192),
            # the other code widths (generic path): 1 bit eight per byte, 5 to 8 bit one per byte
            (1, 64, 1, 16, 512), (1, 32, 0, 24, 100), (5, 32, 1, 20, 256), (6, 64, 0, 64, 96),
-           (7, 16, 1, 8, 64), (8, 64, 1, 33, 192)]
+           (7, 16, 1, 8, 64), (8, 64, 1, 33, 192),
+           # axis-1 groups that cross rows (cols % g != 0): the generic path
+           (4, 64, 1, 40, 96), (2, 32, 1, 30, 48)]
 
 
 @pytest.mark.parametrize("nbits,g,axis,rows,cols", LAYOUTS, ids=lambda v: str(v))

@@ -274,6 +274,123 @@ __global__ void __launch_bounds__(256) hqq_gemv_kernel(const uint32_t *__restric
     if (lane == 0) y[row] = s;
 }
 
+// Axis 1, 2- or 4-bit, group size a multiple of 32 dividing cols: the same product, laid out so
+// that the ALU work, not memory latency, sets the pace.  A piece is 32 consecutive codes of a
+// row (16 bytes of 4-bit codes, 8 of 2-bit), inside one group.  Each warp takes two rows; lane l
+// takes pieces l, l + 32, .. of both (one warp load covers 512 or 256 contiguous bytes), and
+// loads kGv2U pieces of each row with their scale and zero point before using any, then reads
+// the piece's 32 values of x once for both rows.  Two CTAs of eight warps per SM: a 4096-row
+// matrix runs in one wave.
+constexpr int kGv2Rows = 2;
+constexpr int kGv2U = 4;
+
+// dot product of one piece (NB words of codes, one group) with its 32 values of x (xs: 16 fp16
+// pairs), each W_hat value exactly hqq_dequantize's, accumulated in binary32 pairs
+template <int NB>
+__device__ __forceinline__ float2 gemv_piece(const uint32_t *cw, float zf, float df, const uint32_t *xs,
+                                             float2 acc) {
+    const float2 nm = make_float2(-8388608.0f, -8388608.0f), nz = make_float2(-zf, -zf);
+    const float2 d2 = make_float2(df, df);
+#pragma unroll
+    for (int wi = 0; wi < NB; ++wi) {
+        const uint32_t w = cw[wi];
+        if constexpr (NB == 4) {  // word wi: codes 8 wi .. 8 wi + 7, codes 2i, 2i+1 in byte i
+            const uint32_t ev = w & 0x0F0F0F0Fu, od = (w >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 q = make_float2(__uint_as_float(__byte_perm(ev, 0x4B000000u, 0x7540u + i)),
+                                             __uint_as_float(__byte_perm(od, 0x4B000000u, 0x7540u + i)));
+                const float2 v = __fmul2_rn(__fadd2_rn(__fadd2_rn(q, nm), nz), d2);
+                const float2 xf = __half22float2(*reinterpret_cast<const __half2 *>(&xs[4 * wi + i]));
+                acc = __ffma2_rn(__half22float2(__floats2half2_rn(v.x, v.y)), xf, acc);
+            }
+        } else {  // word wi: codes 16 wi .. 16 wi + 15; field s of byte b is code 4b + s
+            uint32_t f[4];
+#pragma unroll
+            for (int s = 0; s < 4; ++s) f[s] = (w >> (2 * s)) & 0x03030303u;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int b = i >> 1, s = 2 * (i & 1);
+                const float2 q = make_float2(__uint_as_float(__byte_perm(f[s], 0x4B000000u, 0x7540u + b)),
+                                             __uint_as_float(__byte_perm(f[s + 1], 0x4B000000u, 0x7540u + b)));
+                const float2 v = __fmul2_rn(__fadd2_rn(__fadd2_rn(q, nm), nz), d2);
+                const float2 xf = __half22float2(*reinterpret_cast<const __half2 *>(&xs[8 * wi + i]));
+                acc = __ffma2_rn(__half22float2(__floats2half2_rn(v.x, v.y)), xf, acc);
+            }
+        }
+    }
+    return acc;
+}
+
+// gshift >= 0: pieces per group 2^gshift; else gpp pieces per group
+template <int NB>
+__global__ void __launch_bounds__(256, 2) hqq_gemv2_kernel(const uint8_t *__restrict__ packed,
+                                                           const __half *__restrict__ scale,
+                                                           const __half *__restrict__ zero,
+                                                           int64_t rows, int ppr, int gshift, int gpp,
+                                                           const __half *__restrict__ x,
+                                                           float *__restrict__ y) {
+    constexpr int PB = 4 * NB;  // bytes per piece
+    const int lane = threadIdx.x & 31;
+    const int64_t r0 = ((int64_t)blockIdx.x * 8 + (threadIdx.x >> 5)) * kGv2Rows;
+    wait_prerequisite();  // codes and x may come from the kernel launched just before
+    allow_dependents();
+    if (r0 >= rows) return;  // whole warps
+    const int64_t gpr = gshift >= 0 ? (int64_t)(ppr >> gshift) : (int64_t)(ppr / gpp);  // groups per row
+    float2 acc[kGv2Rows];
+#pragma unroll
+    for (int r = 0; r < kGv2Rows; ++r) acc[r] = make_float2(0.0f, 0.0f);
+    for (int p0 = lane; p0 < ppr; p0 += 32 * kGv2U) {
+        uint32_t cw[kGv2Rows][kGv2U][NB];
+        float zf[kGv2Rows][kGv2U], df[kGv2Rows][kGv2U];
+#pragma unroll
+        for (int r = 0; r < kGv2Rows; ++r) {
+#pragma unroll
+            for (int i = 0; i < kGv2U; ++i) {
+                const int p = p0 + 32 * i;
+#pragma unroll
+                for (int wi = 0; wi < NB; ++wi) cw[r][i][wi] = 0u;
+                zf[r][i] = 0.0f;
+                df[r][i] = 0.0f;
+                if (p < ppr && r0 + r < rows) {  // absent pieces: codes 0, z = Delta = 0: zero terms
+                    const uint8_t *src = packed + ((r0 + r) * ppr + p) * PB;
+                    if constexpr (NB == 4) {
+                        const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(src));
+                        cw[r][i][0] = v.x; cw[r][i][1] = v.y; cw[r][i][2] = v.z; cw[r][i][3] = v.w;
+                    } else {
+                        const uint2 v = __ldcs(reinterpret_cast<const uint2 *>(src));
+                        cw[r][i][0] = v.x; cw[r][i][1] = v.y;
+                    }
+                    const int64_t k = (r0 + r) * gpr + (gshift >= 0 ? (p >> gshift) : p / gpp);
+                    zf[r][i] = __half2float(__ldg(zero + k));
+                    df[r][i] = __half2float(__ldg(scale + k));
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kGv2U; ++i) {
+            const int p = p0 + 32 * i;
+            if (p < ppr) {
+                uint32_t xs[16];
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(x + (int64_t)p * 32) + v);
+                    xs[4 * v] = xv.x; xs[4 * v + 1] = xv.y; xs[4 * v + 2] = xv.z; xs[4 * v + 3] = xv.w;
+                }
+#pragma unroll
+                for (int r = 0; r < kGv2Rows; ++r) acc[r] = gemv_piece<NB>(cw[r][i], zf[r][i], df[r][i], xs, acc[r]);
+            }
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < kGv2Rows; ++r) {
+        float s = __fadd_rn(acc[r].x, acc[r].y);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) s = __fadd_rn(s, __shfl_xor_sync(kFull, s, off));
+        if (lane == 0 && r0 + r < rows) y[r0 + r] = s;
+    }
+}
+
 // Any other layout: one warp per output row, each lane takes columns lane, lane + 32, ...
 // and reads its codes one at a time (flat row-major code order, groups by axis).
 template <int NB>
@@ -317,8 +434,16 @@ cudaError_t launch_gemv_nb(const uint8_t *pk, const __half *sc, const __half *ze
     constexpr int CPW = Pack<NB>::cpw;
     const unsigned blocks = (unsigned)((rows + 7) / 8);
     const int64_t wpr = cols / CPW;
-    if constexpr (NB == 2 || NB == 4) {  // the fast path: 2- and 4-bit axis-1 layouts
-        // groups must not cross rows (cols % g == 0): the kernel finds a word's group by row
+    if constexpr (NB == 2 || NB == 4) {  // the fast paths: 2- and 4-bit axis-1 layouts
+        // groups must not cross rows (cols % g == 0): the kernels find a word's group by row
+        if (axis == 1 && g % 32 == 0 && cols % g == 0 && ((uintptr_t)x & 15) == 0 && ((uintptr_t)pk & 15) == 0 &&
+            cols / 32 < ((int64_t)1 << 30)) {
+            const int gpp = (int)(g / 32);
+            int shift = -1;
+            if ((gpp & (gpp - 1)) == 0) { shift = 0; while ((1 << shift) < gpp) ++shift; }
+            const unsigned b2 = (unsigned)((rows + 8 * kGv2Rows - 1) / (8 * kGv2Rows));
+            return launch_pdl(hqq_gemv2_kernel<NB>, b2, 256, 0, st, pk, sc, ze, rows, (int)(cols / 32), shift, gpp, x, y);
+        }
         if (axis == 1 && cols % CPW == 0 && g % CPW == 0 && cols % g == 0 && ((uintptr_t)x & 15) == 0 &&
             wpr < ((int64_t)1 << 30)) {
             const int wpg = (int)(g / CPW);

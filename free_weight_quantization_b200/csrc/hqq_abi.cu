@@ -250,6 +250,24 @@ extern "C" int hqq_gemm(const void *packed, const void *scale, const void *zero,
     return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
 }
 
+namespace {
+__global__ void __launch_bounds__(256) hqq_shrink_kernel(const float *__restrict__ r, int64_t n, double beta,
+                                                         double p, float *__restrict__ out) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        out[i] = shrink_lp(r[i], beta, p);
+}
+}  // namespace
+
+extern "C" int hqq_shrink_lp(const float *r, int64_t n, double beta, double p, float *out, void *stream) {
+    if (n < 0 || !(beta > 0.0) || !(p > 0.0)) return HQQ_ERR_ARG;
+    if (n == 0) return HQQ_OK;
+    if (!r || !out) return HQQ_ERR_ARG;
+    if (!aligned_to(r, 4) || !aligned_to(out, 4)) return HQQ_ERR_ALIGN;
+    const unsigned blocks = (unsigned)std::min<int64_t>((n + 255) / 256, 148 * 32);
+    hqq_shrink_kernel<<<blocks, 256, 0, (cudaStream_t)stream>>>(r, n, beta, p, out);
+    return cudaGetLastError() == cudaSuccess ? HQQ_OK : HQQ_ERR_CUDA;
+}
+
 extern "C" const char *hqq_strerror(int code) {
     switch (code) {
     case HQQ_OK: return "ok";

@@ -46,6 +46,7 @@ SIGNATURES = {
                                     _P, _P, _P, _P, _P, _P, _P, _P]),
     "hqq_gemv": (_I32, [_P, _P, _P, _I64, _I64, _I32, _I64, _I32, _P, _P, _P]),
     "hqq_gemm": (_I32, [_P, _P, _P, _I64, _I64, _I32, _I64, _I32, _P, _I64, _P, _P]),
+    "hqq_shrink_lp": (_I32, [_P, _I64, ctypes.c_double, ctypes.c_double, _P, _P]),
     "hqq_strerror": (ctypes.c_char_p, [_I32]),
 }
 
@@ -166,13 +167,20 @@ def hqq_quantize_noalloc(W: torch.Tensor, nbits: int = 4, group_size: int = 64, 
     if W.dtype != torch.float16 or not W.is_cuda or W.dim() != 2 or not W.is_contiguous():
         raise HqqError("W must be a contiguous 2-D float16 CUDA tensor")
     rows, cols = W.shape
+    bufs = [out.packed, out.scale, out.zero, out.iters_run, out.s, out.z, out.err_trace, out.rounds]
+    if any(t is not None and t.device != W.device for t in bufs):
+        raise HqqError("hqq_quantize_noalloc: every output must live on W's device")
     opt = HqqOpt(iters, lp_norm, beta, kappa, eps_tiny, scale_max)
     st = stream if stream is not None else torch.cuda.current_stream(W.device)
-    rc = lib().hqq_quantize_noalloc(_ptr(W), rows, cols, nbits, group_size, axis,
-                                    ctypes.byref(opt), _ptr(out.packed), _ptr(out.scale),
-                                    _ptr(out.zero), _ptr(out.iters_run), _ptr(out.s), _ptr(out.z),
-                                    _ptr(out.err_trace), _ptr(out.rounds),
-                                    ctypes.c_void_p(st.cuda_stream))
+    if st.device != W.device:
+        raise HqqError("hqq_quantize_noalloc: the stream must belong to W's device")
+    # the library finds its scratch buffer on the calling thread's current device
+    with torch.cuda.device(W.device):
+        rc = lib().hqq_quantize_noalloc(_ptr(W), rows, cols, nbits, group_size, axis,
+                                        ctypes.byref(opt), _ptr(out.packed), _ptr(out.scale),
+                                        _ptr(out.zero), _ptr(out.iters_run), _ptr(out.s), _ptr(out.z),
+                                        _ptr(out.err_trace), _ptr(out.rounds),
+                                        ctypes.c_void_p(st.cuda_stream))
     if rc == 3:
         raise HqqError("hqq_quantize_noalloc: this problem needs "
                        f"{hqq_quantize_workspace_bytes(rows, cols, nbits, group_size, axis, iters)}"
@@ -221,6 +229,22 @@ def hqq_gemm(q: Quantized, X: torch.Tensor, out: torch.Tensor | None = None,
     rc = lib().hqq_gemm(_ptr(q.packed), _ptr(q.scale), _ptr(q.zero), q.rows, q.cols, q.nbits,
                         q.group_size, q.axis, _ptr(X), batch, _ptr(out), ctypes.c_void_p(st.cuda_stream))
     _check(rc, "hqq_gemm")
+    return out
+
+
+def hqq_shrink_lp(r: torch.Tensor, beta: float, p: float = 0.7, out: torch.Tensor | None = None,
+                  stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """The proximal step's lp shrink of binary32 residuals, as the quantizer evaluates it (see
+    hqq_shrink_lp in the header)."""
+    if r.dtype != torch.float32 or not r.is_cuda or not r.is_contiguous():
+        raise HqqError("r must be a contiguous float32 CUDA tensor")
+    if out is None:
+        out = torch.empty_like(r)
+    st = stream if stream is not None else torch.cuda.current_stream(r.device)
+    with torch.cuda.device(r.device):
+        rc = lib().hqq_shrink_lp(_ptr(r), r.numel(), float(beta), float(p), _ptr(out),
+                                 ctypes.c_void_p(st.cuda_stream))
+    _check(rc, "hqq_shrink_lp")
     return out
 
 

@@ -185,15 +185,30 @@ int hqq_gemm(const void *packed, const void *scale, const void *zero, int64_t ro
  * library (HQQ_NOALLOC_SCRATCH_BYTES): every GPU that loads the library keeps it until the
  * process exits.  Arguments, outputs and results are those of hqq_quantize; additionally it
  * returns HQQ_ERR_WORKSPACE, launching nothing, when hqq_quantize_workspace_bytes() for these
- * arguments exceeds that buffer.  It allocates nothing.  The first call on each device looks up
- * the buffer's device address (make it before any stream capture).  All calls share the one
- * buffer: calls whose GPU work overlaps (other streams, other host threads) race on it.
+ * arguments exceeds that buffer.  It allocates nothing.  The buffer used is the one of the
+ * calling thread's current device, in that device's primary context (the CUDA runtime's
+ * default; a context made with the driver API is not supported): W, the outputs and the stream
+ * must belong to that device.  The first call on each device looks up the buffer's device
+ * address (make it before any stream capture).  All calls share the one buffer: calls whose GPU
+ * work overlaps (other streams, other host threads) race on it.
  */
 #define HQQ_NOALLOC_SCRATCH_BYTES (4u << 20)
 int hqq_quantize_noalloc(const void *W, int64_t rows, int64_t cols, int nbits, int64_t group_size,
                          int axis, const hqq_opt_t *opt, void *packed, void *scale, void *zero,
                          int32_t *iters_run, float *s_f32, float *z_f32, uint64_t *err_trace,
                          uint8_t *group_rounds, void *stream);
+
+/*
+ * The generalized lp shrink operator of the proximal step [HQQ 算法解读, "shrink 不是删除极值"],
+ * element by element, exactly as hqq_quantize evaluates it inside its rounds:
+ *     out[i] = sign(r[i]) * max(|r[i]| - |r[i]|^(p - 1) / beta, 0)
+ * computed in binary64 from the binary32 r[i] and rounded once to binary32 (0 for r[i] = 0).
+ * r and out: device pointers to n binary32 values (4-byte aligned; out may equal r).  It lets a
+ * caller check the operator against another implementation (the power function is CUDA's).
+ * Returns HQQ_OK (n = 0: nothing launched), HQQ_ERR_ARG (n < 0, beta <= 0, p <= 0, null
+ * pointer), HQQ_ERR_ALIGN or HQQ_ERR_CUDA.
+ */
+int hqq_shrink_lp(const float *r, int64_t n, double beta, double p, float *out, void *stream);
 
 /* Text for a return code (static storage). */
 const char *hqq_strerror(int code);

@@ -74,6 +74,8 @@ def _declare(lib):
     lib.hqo_minmax_init.restype = None
     lib.hqo_shrink.argtypes = [f32, f64, f64]
     lib.hqo_shrink.restype = f32
+    lib.hqo_shrink_n.argtypes = [P, i64, f64, f64, P]
+    lib.hqo_shrink_n.restype = None
     lib.hqo_pairwise_sum.argtypes = [P, i64]
     lib.hqo_pairwise_sum.restype = f32
     lib.hqo_group_pass.argtypes = [P, i64, i32, f32, f32, f64, f64, P, P, P]
@@ -120,6 +122,14 @@ def float_to_half(f: float) -> int:
 
 def shrink(r: float, beta: float, p: float) -> float:
     return _load().hqo_shrink(float(r), float(beta), float(p))
+
+
+def shrink_array(r, beta: float, p: float) -> np.ndarray:
+    """shrink() of every element of a float32 array."""
+    r = np.ascontiguousarray(r, dtype=np.float32)
+    out = np.empty_like(r)
+    _load().hqo_shrink_n(_ptr(r), r.size, float(beta), float(p), _ptr(out))
+    return out
 
 
 def pairwise_sum(x) -> float:

@@ -154,6 +154,13 @@ float hqo_shrink(float r, double beta, double p)
     return r < 0.0f ? -mf : mf;
 }
 
+/* hqo_shrink over an array (test convenience: one call instead of n). */
+void hqo_shrink_n(const float *r, int64_t n, double beta, double p, float *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = hqo_shrink(r[i], beta, p);
+}
+
 /* Pairwise sum of x[lo .. lo+len) with len a power of two; slots at or beyond n are +0. */
 static float pairwise(const float *x, int64_t n, int64_t lo, int64_t len)
 {

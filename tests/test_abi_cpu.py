@@ -153,3 +153,22 @@ def test_binding_arity_matches_the_header():
     for name, params in protos.items():
         n = 0 if params.strip() in ("", "void") else params.count(",") + 1
         assert n == len(hqq.SIGNATURES[name][1]), (name, n, len(hqq.SIGNATURES[name][1]))
+
+
+def test_shrink_rejects_bad_arguments(L):
+    # host-side checks only: nothing reaches a device
+    assert L.hqq_shrink_lp(None, 0, 10.0, 0.7, None, None) == 0
+    assert L.hqq_shrink_lp(None, -1, 10.0, 0.7, None, None) == 1
+    assert L.hqq_shrink_lp(ctypes.c_void_p(16), 4, 0.0, 0.7, ctypes.c_void_p(16), None) == 1
+    assert L.hqq_shrink_lp(ctypes.c_void_p(16), 4, 10.0, 0.0, ctypes.c_void_p(16), None) == 1
+    assert L.hqq_shrink_lp(None, 4, 10.0, 0.7, None, None) == 1
+    assert L.hqq_shrink_lp(ctypes.c_void_p(18), 4, 10.0, 0.7, ctypes.c_void_p(16), None) == 2
+
+
+def test_noalloc_scratch_size_binding_matches_the_header():
+    import os
+    import re
+    text = open(os.path.join(ROOT, "include", "hqq_b200.h")).read()
+    m = re.search(r"#define\s+HQQ_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", text)
+    assert m, "HQQ_NOALLOC_SCRATCH_BYTES not found in the header"
+    assert hqq.HQQ_NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))

@@ -169,6 +169,15 @@ def test_shrink_lp_shape():
         assert all(b >= a for a, b in zip(es, es[1:]))
 
 
+def test_shrink_array_is_the_scalar_shrink():
+    # the array form used by the GPU agreement check is the scalar operator, element by element
+    r = np.random.default_rng(5).standard_normal(2000).astype(np.float32) * 0.5
+    for beta in [10.0, 10.0 * 1.01 ** 19]:
+        got = oracle.shrink_array(r, beta, 0.7)
+        want = np.array([oracle.shrink(float(v), beta, 0.7) for v in r], np.float32)
+        assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+
+
 # ------------------------------------------------------------------ one proximal pass
 @pytest.mark.parametrize("g,nbits", [(4, 2), (5, 3), (8, 4), (6, 4)])
 def test_zero_update_is_least_squares(g, nbits):

@@ -26,12 +26,12 @@ def hqq():
     return h
 
 
-def _outputs(h, rows, cols, nbits, g, iters):
+def _outputs(h, rows, cols, nbits, g, iters, axis=1):
     N, G = rows * cols, rows * cols // g
     dev = "cuda"
     return h.Quantized(torch.empty(max(oracle.packed_bytes(N, nbits), 1), dtype=torch.uint8, device=dev),
                        torch.empty(G, dtype=torch.float16, device=dev),
-                       torch.empty(G, dtype=torch.float16, device=dev), rows, cols, nbits, g, 1,
+                       torch.empty(G, dtype=torch.float16, device=dev), rows, cols, nbits, g, axis,
                        torch.zeros(1, dtype=torch.int32, device=dev),
                        torch.empty(G, dtype=torch.float32, device=dev),
                        torch.empty(G, dtype=torch.float32, device=dev),
@@ -46,6 +46,16 @@ def _same(a, b):
                            y.view(torch.uint8) if y.dtype == torch.float16 else y), f
     n = int(a.iters_run.item())
     assert torch.equal(a.err_trace[:2 * n], b.err_trace[:2 * n])
+
+
+def _matches_oracle(h, q, Wn, nbits, g, axis):
+    o = oracle.quantize(Wn, nbits, g, axis)
+    n = int(q.iters_run.item())
+    assert n == o["iters_run"]
+    assert h.err_trace_ints(q.err_trace, n) == o["err_trace"]
+    assert np.array_equal(q.packed.cpu().numpy()[:o["packed"].size], o["packed"])
+    assert np.array_equal(q.scale.cpu().numpy().view(np.uint16), o["scale"].view(np.uint16))
+    assert np.array_equal(q.zero.cpu().numpy().view(np.uint16), o["zero"].view(np.uint16))
 
 
 @pytest.mark.parametrize("case", [wl.SMALL, wl.MLP_B2], ids=lambda c: c.name)
@@ -63,6 +73,24 @@ def test_noalloc_matches_workspace_entry_point_twice(hqq, case):
         if i > 0:  # after the first call (which may load the library's module) nothing grows
             assert torch.cuda.mem_get_info()[0] == free_before
         _same(ref, out)
+        if rows * cols <= 1 << 20:  # and both are the oracle's result
+            _matches_oracle(hqq, out, np.ascontiguousarray(Wn), case.nbits, case.group_size, 1)
+
+
+# the tile engine's paths: 3-bit codes; axis 0 with a group count (300) that is not a multiple
+# of the 8 codes of a packed word, so that the codes go through byte staging in the scratch
+@pytest.mark.parametrize("rows,cols,nbits,g,axis", [(64, 640, 3, 64, 1), (128, 300, 4, 128, 0)],
+                         ids=["3bit-g64", "axis0-g128-G300"])
+def test_noalloc_tile_paths_twice(hqq, rows, cols, nbits, g, axis):
+    assert hqq.hqq_quantize_workspace_bytes(rows, cols, nbits, g, axis, 20) <= hqq.HQQ_NOALLOC_SCRATCH_BYTES
+    out = _outputs(hqq, rows, cols, nbits, g, 20, axis)
+    for Wn in [wl.student_t(rows, cols, seed=5), wl.outlier_normal(rows, cols, seed=6)]:
+        W = torch.from_numpy(np.ascontiguousarray(Wn)).cuda()
+        ref = hqq.hqq_quantize(W, nbits, g, axis, iters=20, debug=True)
+        hqq.hqq_quantize_noalloc(W, nbits, g, axis, iters=20, out=out)
+        torch.cuda.synchronize()
+        _same(ref, out)
+        _matches_oracle(hqq, out, np.ascontiguousarray(Wn), nbits, g, axis)
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(hqq):

@@ -17,7 +17,9 @@ hqq_dequantize.  Inputs rotate over enough copies that every step reads its matr
   - `e2e`: the same metric through the public API with pinned host buffers, copies included;
   - `cpu_baseline`: the CPU oracle on the host, on all cores (OpenMP timing build) and on one;
   - `dequant_back_to_back` and `gemv`: dequantize and the fused forward product, each timed
-    back to back by CUDA-graph replay, with the unfused dequantize + matmul beside the latter.
+    back to back by CUDA-graph replay, with the unfused dequantize + matmul beside the latter;
+  - `gemm`: the batched forward product (tensor cores) for batches 1, 16, 64 and 256, timed
+    the same way, beside the unfused dequantize + matmul.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                   [--workload attn|small|mlp_b2|mlp_b3|attn_ax0|stack] [--no-per-config]
@@ -697,6 +699,32 @@ def main():
     gemv_ms, _ = rig.per_call_ms(loop_gemv, nb2b)
     unfused_ms, _ = rig.per_call_ms(loop_unfused, nb2b)
 
+    # The batched forward product Y = X @ W_hat.T (hqq_gemm: the tcgen05 tensor-core kernel on
+    # this layout) for a few batch sizes, beside the unfused dequantize + library fp16 matmul.
+    gemm = {}
+    for batch in (1, 16, 64, 256):
+        Xb = torch.randn(batch, COLS, device=dev).to(torch.float16)
+        Yb = [torch.empty(batch, ROWS, dtype=torch.float32, device=dev) for _ in range(rig.rotate)]
+        Yh = [torch.empty(batch, ROWS, dtype=torch.float16, device=dev) for _ in range(rig.rotate)]
+
+        def loop_gemm(n, Xb=Xb, Yb=Yb):
+            for i in range(n):
+                hqq.hqq_gemm(rig.outs[i % rig.rotate], Xb, out=Yb[i % rig.rotate])
+
+        def loop_gemm_unfused(n, Xb=Xb, Yh=Yh):
+            for i in range(n):
+                k = i % rig.rotate
+                rig.dequantize(i)
+                torch.matmul(Xb, rig.deqs[k].t(), out=Yh[k])
+
+        ng = max(2 * rig.rotate, min(K, 200))
+        g_ms, _ = rig.per_call_ms(loop_gemm, ng)
+        u_ms, _ = rig.per_call_ms(loop_gemm_unfused, ng)
+        gb = packed_bytes + 4 * G + 2 * batch * COLS + 4 * batch * ROWS
+        gemm[str(batch)] = {"us": g_ms * 1e3, "tflops": 2 * ROWS * COLS * batch / (g_ms / 1e3) / 1e12,
+                            "gbs": gb / (g_ms / 1e3) / 1e9, "alg_bytes_per_launch": gb,
+                            "unfused_dequant_then_matmul_us": u_ms * 1e3}
+
     # end to end through the public API: pinned host W in, packed codes + metadata + dequantized
     # W out, copies inside the timed region.  Two slots, each with its own stream, device
     # buffers, workspace and pinned host outputs, alternate steps, so one step's upload overlaps
@@ -800,6 +828,8 @@ def main():
                      "alg_bytes_per_launch": packed_bytes + 4 * G + 2 * COLS + 4 * ROWS,
                      "unfused_dequant_then_matmul_us": unfused_ms * 1e3, "launches": nb2b,
                      "timed_by": b2b_how},
+            "gemm": {"batches": gemm, "timed_by": b2b_how,
+                     "kernel": "tcgen05 (A = dequantized W from tensor memory, B = X by TMA)"},
             "hbm_peak_gbs": pk["hbm_gbs"], "hbm_peak_src": pk["src"],
             "alg_bytes_per_launch": alg_bytes,
             "roofline": roofline,

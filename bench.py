@@ -720,7 +720,7 @@ def main():
         ng = max(2 * rig.rotate, min(K, 200))
         g_ms, _ = rig.per_call_ms(loop_gemm, ng)
         u_ms, _ = rig.per_call_ms(loop_gemm_unfused, ng)
-        gb = packed_bytes + 4 * G + 2 * batch * COLS + 4 * batch * ROWS
+        gb = rig.packed_bytes + 4 * G + 2 * batch * COLS + 4 * batch * ROWS
         gemm[str(batch)] = {"us": g_ms * 1e3, "tflops": 2 * ROWS * COLS * batch / (g_ms / 1e3) / 1e12,
                             "gbs": gb / (g_ms / 1e3) / 1e9, "alg_bytes_per_launch": gb,
                             "unfused_dequant_then_matmul_us": u_ms * 1e3}

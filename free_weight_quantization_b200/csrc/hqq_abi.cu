@@ -239,9 +239,10 @@ extern "C" int hqq_gemm(const void *packed, const void *scale, const void *zero,
     const uint8_t *pk = (const uint8_t *)packed;
     const __half *sc = (const __half *)scale, *ze = (const __half *)zero, *xh = (const __half *)X;
     cudaError_t e;
-    if (hqq_impl::gemm_tc_layout(nbits, rows, cols, pl.g, axis, X)) {
+    // one input vector: the SIMT product is faster than four N = 16 MMAs per tile
+    if (batch >= 2 && hqq_impl::gemm_tc_layout(nbits, rows, cols, pl.g, axis, X)) {
         e = hqq_impl::launch_gemm_tc(nbits, pk, sc, ze, rows, cols, pl.g, xh, batch, Y, st);
-    } else {  // any other layout: the generic product, one batch entry at a time
+    } else {  // a single vector, or any other layout: the one-vector product per batch entry
         e = cudaSuccess;
         for (int64_t b = 0; b < batch && e == cudaSuccess; ++b)
             e = hqq_impl::launch_gemv(nbits, pk, sc, ze, rows, cols, pl.g, pl.G, axis, xh + b * cols,

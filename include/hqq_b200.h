@@ -169,8 +169,8 @@ int hqq_gemv(const void *packed, const void *scale, const void *zero, int64_t ro
  *   stream  cudaStream_t, or NULL for the default stream
  * Axis-1 layouts with 2- or 4-bit codes, group_size a multiple of 8 that divides cols, cols a
  * multiple of 64 and a 16-byte aligned X run on the tensor cores (tcgen05.mma, fp16 operands, binary32 accumulators in
- * tensor memory; up to 256 batch entries per launch).  Every other layout runs the one-vector
- * product once per batch entry.
+ * tensor memory; up to 256 batch entries per launch) when batch >= 2.  A batch of one, and
+ * every other layout, runs the one-vector product (hqq_gemv) once per batch entry.
  * Returns HQQ_OK, HQQ_ERR_ARG (shape, batch or null pointer), HQQ_ERR_ALIGN, or HQQ_ERR_CUDA.
  */
 int hqq_gemm(const void *packed, const void *scale, const void *zero, int64_t rows, int64_t cols,

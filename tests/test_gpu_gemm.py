@@ -4,7 +4,8 @@ W_hat is the fp16 dequantized weight in both.  Each product of two fp16 values i
 binary32, so the GPU result differs from the exact sum only by its binary32 accumulation,
 whatever its order or the tensor cores' rounding of partial sums: the check allows
 cols * 2^-23 * sum_c |W_hat x| per element.  Axis-1 2- and 4-bit layouts with cols a multiple
-of 64 run the tcgen05 tensor-core kernel; the rest the generic product per batch entry.
+of 64 run the tcgen05 tensor-core kernel when the batch has two entries or more; a batch of one
+and the other layouts the one-vector product per batch entry.
 """
 import numpy as np
 import pytest
@@ -43,7 +44,7 @@ def _check(Y, ref, mag, cols, label):
 # (nbits, group_size, axis, rows, cols, batch): tensor-core layouts first (one tile, split
 # columns, ragged row block, the largest MMA N, more than one launch of batch entries, 2 bit),
 # then layouts on the generic path
-CASES = [(4, 64, 1, 128, 64, 1), (4, 64, 1, 256, 512, 2), (4, 64, 1, 200, 1024, 7),
+CASES = [(4, 64, 1, 128, 64, 2), (4, 64, 1, 128, 64, 1), (4, 64, 1, 256, 512, 2), (4, 64, 1, 200, 1024, 7),
          (4, 128, 1, 384, 2048, 16), (4, 32, 1, 128, 256, 33), (4, 64, 1, 512, 1024, 256),
          (4, 64, 1, 256, 512, 300), (2, 16, 1, 256, 1024, 5), (2, 64, 1, 130, 128, 64),
          (4, 8, 1, 128, 128, 3),
@@ -69,19 +70,19 @@ def test_gemm_random_codes(hqq, nbits, g, axis, rows, cols, batch):
 
 
 def test_gemm_matches_the_one_vector_product_and_batch_zero(hqq):
-    # batch 1 through the tensor cores against the CUDA-core product of the same codes, and an
-    # empty batch launches nothing
-    c = wl.ATTN
+    # a batch of one takes the one-vector product (same bits); a batch of two the tensor cores,
+    # each row within the bound of the oracle's product; an empty batch launches nothing
     W = torch.from_numpy(wl.student_t(512, 1024, seed=4)).cuda()
     q = hqq.hqq_quantize(W, 4, 64, 1)
-    x = torch.randn(1, 1024, device="cuda").to(torch.float16)
-    y1 = hqq.hqq_gemm(q, x)[0].cpu().numpy().astype(np.float64)
-    y2 = hqq.hqq_gemv(q, x[0]).cpu().numpy().astype(np.float64)
-    ref, mag = oracle.gemv(q.packed.cpu().numpy()[:oracle.packed_bytes(512 * 1024, 4)],
-                           q.scale.cpu().numpy(), q.zero.cpu().numpy(), 512, 1024, 4, 64, 1,
-                           x[0].cpu().numpy())
-    for y in (y1, y2):
-        assert (np.abs(y - ref) <= 1024 * 2.0 ** -23 * mag + 1e-30).all()
+    X = torch.randn(2, 1024, device="cuda").to(torch.float16)
+    y1 = hqq.hqq_gemm(q, X[:1])[0].cpu().numpy()
+    assert np.array_equal(y1.view(np.uint32), hqq.hqq_gemv(q, X[0]).cpu().numpy().view(np.uint32))
+    Y2 = hqq.hqq_gemm(q, X).cpu().numpy().astype(np.float64)
+    for b in range(2):
+        ref, mag = oracle.gemv(q.packed.cpu().numpy()[:oracle.packed_bytes(512 * 1024, 4)],
+                               q.scale.cpu().numpy(), q.zero.cpu().numpy(), 512, 1024, 4, 64, 1,
+                               X[b].cpu().numpy())
+        assert (np.abs(Y2[b] - ref) <= 1024 * 2.0 ** -23 * mag + 1e-30).all()
     out = hqq.hqq_gemm(q, torch.empty(0, 1024, dtype=torch.float16, device="cuda"))
     assert out.shape == (0, 512)
 

@@ -49,7 +49,10 @@ LAYOUTS = [(4, 64, 1, 96, 512), (2, 16, 1, 64, 256), (4, 128, 1, 33, 1024), (2, 
            (1, 64, 1, 16, 512), (1, 32, 0, 24, 100), (5, 32, 1, 20, 256), (6, 64, 0, 64, 96),
            (7, 16, 1, 8, 64), (8, 64, 1, 33, 192),
            # axis-1 groups that cross rows (cols % g != 0): the generic path
-           (4, 64, 1, 40, 96), (2, 32, 1, 30, 48)]
+           (4, 64, 1, 40, 96), (2, 32, 1, 30, 48),
+           # 16 MiB of codes and more: the bulk-copy kernel; 8195 rows end in a 3-row stage
+           # whose 195 metadata halves are not whole 16-byte units (65 groups per row)
+           (4, 64, 1, 8195, 4160), (2, 64, 1, 8192, 8192)]
 
 
 @pytest.mark.parametrize("nbits,g,axis,rows,cols", LAYOUTS, ids=lambda v: str(v))

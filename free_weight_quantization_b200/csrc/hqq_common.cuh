@@ -33,6 +33,7 @@ struct QParams {
     int stride;     // floats per group row of the shared tile
     int tile;       // groups per tile
     int stream_warps;  // warps of each stream-engine CTA that take groups (the rest idle)
+    int stream_lanes;  // lanes of such a warp that take groups (32, or 4 for a small tensor)
     int64_t acc_words; // 64-bit words of round sums and control words zeroed before each call
     uint8_t *packed;
     int64_t packed_bytes;

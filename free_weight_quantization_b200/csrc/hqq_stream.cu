@@ -486,8 +486,9 @@ __global__ void __launch_bounds__(kThreads, P <= 64 ? 2 : 1) hqq_stream_kernel(c
     // the round sums and the group counter were zeroed by the kernel launched before this one
     wait_prerequisite();
     // a small tensor is spread thin: only the first stream_warps warps of each CTA take groups,
-    // so its few groups run on many SMs rather than crowding a few
-    int64_t nxt = warp < Pm.stream_warps ? claim(Pm, true) : -1;
+    // so its few groups run on many SMs rather than crowding a few; a very small one also takes
+    // only stream_lanes groups per warp, so that the lane split below starts at once
+    int64_t nxt = warp < Pm.stream_warps ? claim(Pm, lane < Pm.stream_lanes) : -1;
     if (nxt >= 0) prefetch_row<P>(slot, Pm.W, nxt, sw);
     while (true) {
         // ---- a lane without a group takes the prefetched one and prefetches another
@@ -706,8 +707,13 @@ cudaError_t launch_stream(const QParams &Pm, cudaStream_t st) {
     // warps that take groups in each CTA: all of them once the tensor fills the resident grid,
     // fewer (down to one) for a small tensor, so that its groups land on as many SMs as possible
     const int64_t slots = (int64_t)sms * per_sm;
-    const int64_t warps_needed = (Pm.G + 31) / 32;
     QParams Q = Pm;
+    // A tensor whose groups fit the resident grid at kTailLanes per warp runs split from the
+    // start: every group on up to 8 lanes, so that its rounds, which run one after another,
+    // take less time each (256x512 4-bit g64: 2048 groups on 512 warps).
+    Q.stream_lanes = 32;
+    if (TailMax<NB, P>::value >= 2 && Pm.K > 0 && Pm.G <= slots * kWarps * kTailLanes) Q.stream_lanes = kTailLanes;
+    const int64_t warps_needed = (Pm.G + Q.stream_lanes - 1) / Q.stream_lanes;
     Q.stream_warps = (int)std::min<int64_t>(kWarps, std::max<int64_t>(1, (warps_needed + slots - 1) / slots));
     const unsigned blocks = (unsigned)std::max<int64_t>(
         1, std::min<int64_t>(slots, (warps_needed + Q.stream_warps - 1) / Q.stream_warps));

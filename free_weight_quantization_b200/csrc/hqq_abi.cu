@@ -8,13 +8,16 @@
 
 namespace {
 
+// groups up to which a stream-engine tensor keeps its zeros per round (G x iters binary32)
+constexpr int64_t kZringMaxGroups = 16384;
+
 struct Plan {
     int64_t N, G;
     int g, P, L, stride, tile;  // stride: floats per tile row
     int64_t ntiles;
     bool aligned;  // packed words can be written per tile
     bool stream;   // axis 1, 2- or 4-bit, power-of-two groups of 16 .. 128 (the stream engine)
-    size_t ws_acc, ws_fk, ws_tile, ws_stale, ws_codes, ws_total;
+    size_t ws_acc, ws_fk, ws_tile, ws_stale, ws_codes, ws_zring, ws_total;
 };
 
 int64_t gcd64(int64_t a, int64_t b) {
@@ -75,7 +78,10 @@ int make_plan(int64_t rows, int64_t cols, int nbits, int64_t group_size, int axi
     pl->ws_tile = (size_t)((pl->ntiles + 15) / 16 * 16);
     pl->ws_stale = (size_t)(4 * pl->ntiles + 15) / 16 * 16;
     pl->ws_codes = pl->aligned ? 0 : (size_t)((N + 15) / 16 * 16);
-    pl->ws_total = pl->ws_acc + pl->ws_fk + pl->ws_tile + pl->ws_stale + pl->ws_codes;
+    // a small stream-engine tensor keeps every group's zero after each update, so that the
+    // fixup of a stale group reads the kept zero instead of replaying the rounds up to it
+    pl->ws_zring = pl->stream && iters > 0 && pl->G <= kZringMaxGroups ? (size_t)pl->G * iters * 4 : 0;
+    pl->ws_total = pl->ws_acc + pl->ws_fk + pl->ws_tile + pl->ws_stale + pl->ws_codes + pl->ws_zring;
     return HQQ_OK;
 }
 
@@ -161,6 +167,7 @@ extern "C" int hqq_quantize(const void *W, int64_t rows, int64_t cols, int nbits
     P.tile_maxf = wtile;
     P.stale = (int *)(wtile + pl.ws_tile);
     P.codes_u8 = pl.aligned ? nullptr : wtile + pl.ws_tile + pl.ws_stale;
+    P.zring = pl.ws_zring ? (float *)(wtile + pl.ws_tile + pl.ws_stale + pl.ws_codes) : nullptr;
     P.iters_run = iters_run;
     P.err_trace = (u64 *)err_trace;
     P.group_rounds = group_rounds;

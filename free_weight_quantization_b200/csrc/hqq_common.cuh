@@ -44,6 +44,7 @@ struct QParams {
     uint8_t *tile_maxf;  // [ntiles] largest f of each tile
     int *stale;     // [ntiles] tiles holding a group whose last round lies past the kept one
     uint8_t *codes_u8;  // [N] byte-per-code staging when the packed layout is not tile aligned
+    float *zring;       // [G][K] zero after each update (small stream-engine tensors), or null
     int32_t *iters_run;
     u64 *err_trace;
     uint8_t *group_rounds;  // [G] nullable: rounds run by each group in the search kernel

@@ -409,6 +409,7 @@ __device__ void tail_epoch(const QParams &Pm, TailState &ts, unsigned &owners, f
                 if (l == 0) stream_meta(Pm, me.cur, me.gs.s, me.gs.y, me.gs.z, me.it);
                 me.act = false;  // keeps its consistent row and state
             } else {
+                if (l == 0 && Pm.zring) Pm.zring[me.cur * K + me.it] = znew;
                 me.gs.z = znew;
                 ++me.it;
             }
@@ -569,6 +570,7 @@ __global__ void __launch_bounds__(kThreads, P <= 64 ? 2 : 1) hqq_stream_kernel(c
                 add_fixed(acc_w + 4 * it, fx);
                 if (done && it + 1 < K) add_fixed(acc_w + 4 * (K + it + 1), fx);
                 if (!done) {
+                    if (Pm.zring) Pm.zring[cur * K + it] = znew;
                     gs.z = znew;
                     ++it;
                 }
@@ -669,7 +671,9 @@ __global__ void __launch_bounds__(kThreads) hqq_stream_fixup_kernel(const __grid
                 group_init<NB, P>(row, Pm.eps_tiny, Pm.scale_max, gs);
             }
             const int n = stale ? min(b, f) : 0;
-            for (int r = 0; __any_sync(kFull, r < n); ++r) {
+            // with the zeros kept per update, the n-th one is read instead of replayed
+            if (Pm.zring && stale && n > 0) gs.z = __ldcg(Pm.zring + grp * K + (n - 1));
+            for (int r = 0; !Pm.zring && __any_sync(kFull, r < n); ++r) {
                 build_table<NQ>(col, gs.s, gs.y, gs.z);
                 float esum, zsum;
                 SCodes<NB, P, false> nocodes;

@@ -393,7 +393,16 @@ __device__ void tail_epoch(const QParams &Pm, TailState &ts, unsigned &owners, f
         }
         const float B = resid_bound(lz, hz, me.gs.A, me.gs.z, me.gs.y, kQmax);
         const bool slow = me.act && B > thr_s[ri];
-        if (slow) zsum = group_zsum_shrink<NB>(Pm.W + me.cur * P, P, P, me.gs.s, me.gs.z, tab_adj, beta_s[ri], Pm.p);
+        if (__any_sync(kFull, slow)) {
+            // the exact binary64 shrink, each lane over its own slice; the segment's shuffle
+            // levels then continue the halving, the order of the whole-group evaluation
+            float zs = slow ? group_zsum_shrink<NB>(Pm.W + me.cur * P + l * E, E, E, me.gs.s, me.gs.z, tab_adj,
+                                                    beta_s[ri], Pm.p)
+                            : 0.0f;
+#pragma unroll
+            for (int off = 1; off < L; off <<= 1) zs = __fadd_rn(zs, __shfl_xor_sync(kFull, zs, off));
+            if (slow) zsum = zs;
+        }
         const float znew = __fmul_rn(zsum, 1.0f / (float)P);
         if (me.act) {
             const bool done = (!slow && !(B > thr_last) && znew == me.gs.z) || me.it == K - 1;

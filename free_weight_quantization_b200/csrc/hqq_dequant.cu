@@ -276,12 +276,14 @@ __global__ void __launch_bounds__(256) hqq_gemv_kernel(const uint32_t *__restric
 
 // Axis 1, 2- or 4-bit, group size a multiple of 32 dividing cols: the same product, laid out so
 // that the ALU work, not memory latency, sets the pace.  A piece is 32 consecutive codes of a
-// row (16 bytes of 4-bit codes, 8 of 2-bit), inside one group.  Each warp takes two rows; lane l
-// takes pieces l, l + 32, .. of both (one warp load covers 512 or 256 contiguous bytes), and
+// row (16 bytes of 4-bit codes, 8 of 2-bit), inside one group.  Each warp takes kGv2Rows rows;
+// lane l takes pieces l, l + 32, .. (one warp load covers 512 or 256 contiguous bytes), and
 // loads kGv2U pieces of each row with their scale and zero point before using any, then reads
-// the piece's 32 values of x once for both rows.  Two CTAs of eight warps per SM: a 4096-row
-// matrix runs in one wave.
-constexpr int kGv2Rows = 2;
+// the piece's 32 values of x once for all the warp's rows.  One row per warp at 63 registers
+// lets four CTAs of eight warps share an SM, which hides the loads best (4096^2 4-bit, back to
+// back: two rows per warp at two CTAs per SM 9.4 us, two rows at three 11.0 us, one row at
+// four 8.3 us).
+constexpr int kGv2Rows = 1;
 constexpr int kGv2U = 4;
 
 // dot product of one piece (NB words of codes, one group) with its 32 values of x (xs: 16 fp16
@@ -324,7 +326,7 @@ __device__ __forceinline__ float2 gemv_piece(const uint32_t *cw, float zf, float
 
 // gshift >= 0: pieces per group 2^gshift; else gpp pieces per group
 template <int NB>
-__global__ void __launch_bounds__(256, 2) hqq_gemv2_kernel(const uint8_t *__restrict__ packed,
+__global__ void __launch_bounds__(256, 4) hqq_gemv2_kernel(const uint8_t *__restrict__ packed,
                                                            const __half *__restrict__ scale,
                                                            const __half *__restrict__ zero,
                                                            int64_t rows, int ppr, int gshift, int gpp,

@@ -149,6 +149,81 @@ __global__ void __launch_bounds__(kDqThreads) hqq_dequant_kernel(
     }
 }
 
+// 3-bit codes, axis 1, group size >= 40: four packed words (40 codes) per thread and step, so
+// that each thread reads 16 bytes and writes its 80 output bytes with five 16-byte stores
+// (a 10-code word alone is 20 bytes of output, which only 4-byte stores can write).  40
+// consecutive codes touch at most two groups; both metadata pairs are loaded with the words.
+constexpr int kDq3U = 2;
+
+__global__ void __launch_bounds__(kDqThreads) hqq_dequant3_kernel(
+    const uint32_t *__restrict__ packed, const __half *__restrict__ scale,
+    const __half *__restrict__ zero, int64_t N, int g, int64_t G, int gshift,
+    __half *__restrict__ out) {
+    const int64_t nwords = (N + 9) / 10, nunits = (N + 39) / 40;
+    const int64_t ubase = (int64_t)blockIdx.x * (kDqThreads * kDq3U) + threadIdx.x;
+    wait_prerequisite();  // the codes may come from the kernel launched just before
+    allow_dependents();
+    uint32_t wd[kDq3U][4];
+    float z0[kDq3U], d0[kDq3U], z1[kDq3U], d1[kDq3U];
+    int cb[kDq3U];
+#pragma unroll
+    for (int u = 0; u < kDq3U; ++u) {
+        const int64_t t = ubase + u * kDqThreads;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) wd[u][i] = 0u;
+        z0[u] = d0[u] = z1[u] = d1[u] = 0.0f;
+        cb[u] = 40;
+        if (t < nunits) {
+            if (4 * t + 4 <= nwords) {
+                const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(packed) + t);
+                wd[u][0] = v.x; wd[u][1] = v.y; wd[u][2] = v.z; wd[u][3] = v.w;
+            } else {  // the last unit may hold fewer than four words
+                for (int i = 0; i < 4 && 4 * t + i < nwords; ++i) wd[u][i] = __ldcs(packed + 4 * t + i);
+            }
+            const int64_t n0 = 40 * t;
+            const int64_t k0 = gshift >= 0 ? (n0 >> gshift) : n0 / g;
+            const int64_t k1 = k0 + 1 < G ? k0 + 1 : k0;
+            cb[u] = (int)(g - (n0 - k0 * g));  // codes c < cb belong to group k0
+            z0[u] = __half2float(__ldg(zero + k0));
+            d0[u] = __half2float(__ldg(scale + k0));
+            z1[u] = __half2float(__ldg(zero + k1));
+            d1[u] = __half2float(__ldg(scale + k1));
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < kDq3U; ++u) {
+        const int64_t t = ubase + u * kDqThreads;
+        if (t >= nunits) break;
+        const int64_t n0 = 40 * t;
+        uint32_t res[20];
+#pragma unroll
+        for (int c = 0; c < 40; c += 2) {
+            float v[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int cc = c + e;
+                const bool first = cc < cb[u];
+                const uint32_t q = (wd[u][cc / 10] >> (3 * (cc % 10))) & 7u;
+                const float qf = __fsub_rn(__int_as_float(0x4B000000 | (int)q), 8388608.0f);
+                v[e] = __fmul_rn(__fsub_rn(qf, first ? z0[u] : z1[u]), first ? d0[u] : d1[u]);
+            }
+            const __half2 h2 = __floats2half2_rn(v[0], v[1]);
+            memcpy(&res[c / 2], &h2, 4);
+        }
+        if (n0 + 40 <= N) {  // 80 bytes at a multiple of 80: 16-byte aligned
+            uint4 *dst = reinterpret_cast<uint4 *>(out + n0);
+#pragma unroll
+            for (int i = 0; i < 5; ++i)
+                __stcs(dst + i, make_uint4(res[4 * i], res[4 * i + 1], res[4 * i + 2], res[4 * i + 3]));
+        } else {
+            unsigned short *o16 = reinterpret_cast<unsigned short *>(out + n0);
+#pragma unroll
+            for (int c = 0; c < 40; ++c)
+                if (n0 + c < N) o16[c] = (unsigned short)(res[c / 2] >> (16 * (c % 2)));
+        }
+    }
+}
+
 template <int NB>
 cudaError_t launch_dequant(const uint8_t *pk, const __half *sc, const __half *ze, int64_t N, int g,
                     int64_t G, int axis, int64_t pb, __half *out, cudaStream_t st) {
@@ -165,6 +240,13 @@ cudaError_t launch_dequant(const uint8_t *pk, const __half *sc, const __half *ze
     // programmatic launch: overlaps the kernel before it, which the kernel waits for
     if (axis == 1 && g % CPW == 0)
         return launch_pdl(hqq_dequant_kernel<NB, 0>, blocks, kDqThreads, 0, st, pw, sc, ze, N, g, G, pb, shift, false, out);
+    if (NB == 3 && axis == 1 && g >= 40 && ((uintptr_t)pk & 15) == 0 && ((uintptr_t)out & 15) == 0) {
+        int gs = -1;
+        if ((g & (g - 1)) == 0) { gs = 0; while ((1 << gs) < g) ++gs; }
+        const int64_t nunits = (N + 39) / 40;
+        const unsigned b3 = (unsigned)((nunits + kDqThreads * kDq3U - 1) / (kDqThreads * kDq3U));
+        return launch_pdl(hqq_dequant3_kernel, b3, kDqThreads, 0, st, pw, sc, ze, N, g, G, gs, out);
+    }
     if (axis == 1 && g >= CPW) {  // a word spans at most two groups
         int gs = -1;
         if ((g & (g - 1)) == 0) { gs = 0; while ((1 << gs) < g) ++gs; }

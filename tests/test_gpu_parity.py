@@ -153,7 +153,10 @@ def test_full_size_config(case, pool):
 @pytest.mark.parametrize("nbits", [1, 2, 3, 4, 5, 6, 7, 8])
 @pytest.mark.parametrize("shape,g,axis", [((64, 64), 64, 1), ((37, 129), 3, 1), ((100, 7), 10, 1),
                                           ((256, 64), 128, 0), ((30, 32), 16, 0),
-                                          ((41, 40), 8, 0)])
+                                          ((41, 40), 8, 0),
+                                          # 3-bit, groups of 40 and more: four words per thread,
+                                          # groups that straddle them, a ragged last unit
+                                          ((33, 200), 40, 1), ((7, 130), 65, 1), ((96, 160), 96, 1)])
 def test_dequant_random_codes(nbits, shape, g, axis):
     from free_weight_quantization_b200 import hqq
     rows, cols = shape

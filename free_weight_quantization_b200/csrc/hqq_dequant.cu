@@ -224,6 +224,56 @@ __global__ void __launch_bounds__(kDqThreads) hqq_dequant3_kernel(
     }
 }
 
+// Axis 0 with g dividing rows (and CPW = 8: 4-bit codes): element n is in group n mod G and G is
+// a whole number of rows, so the metadata of a word's 8 groups repeats every G elements.  A
+// thread owns one such word position j (elements 8 j .. 8 j + 7 of each G-element stripe),
+// loads its 8 scale/zero pairs once (two 16-byte loads) and dequantizes kDqA0M of the g words
+// at j, j + G/8, ...; consecutive threads take consecutive words, so loads and 16-byte stores
+// stay coalesced.  (The general axis-0 path reloads the metadata for every word: four bytes of
+// metadata per weight from L2, twice the output's bytes.)
+constexpr int kDqA0M = 16;
+
+__global__ void __launch_bounds__(kDqThreads) hqq_dequant_a0_kernel(
+    const uint32_t *__restrict__ packed, const __half *__restrict__ scale,
+    const __half *__restrict__ zero, int64_t G, int g, __half *__restrict__ out) {
+    const int64_t wpg = G / 8;  // words per stripe
+    const int64_t t = (int64_t)blockIdx.x * kDqThreads + threadIdx.x;
+    const int64_t j = t % wpg, m0 = (t / wpg) * kDqA0M;
+    wait_prerequisite();  // the codes may come from the kernel launched just before
+    allow_dependents();
+    if (m0 >= g) return;
+    const uint4 zv = __ldg(reinterpret_cast<const uint4 *>(zero + 8 * j));
+    const uint4 dv = __ldg(reinterpret_cast<const uint4 *>(scale + 8 * j));
+    const __half *zh = reinterpret_cast<const __half *>(&zv), *dh = reinterpret_cast<const __half *>(&dv);
+    float zf[8], df[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        zf[c] = __half2float(zh[c]);
+        df[c] = __half2float(dh[c]);
+    }
+    const int mend = m0 + kDqA0M < g ? (int)m0 + kDqA0M : g;
+    uint32_t wd[kDqA0M];
+#pragma unroll
+    for (int i = 0; i < kDqA0M; ++i) wd[i] = (int)m0 + i < mend ? __ldcs(packed + (m0 + i) * wpg + j) : 0u;
+#pragma unroll
+    for (int i = 0; i < kDqA0M; ++i) {
+        if ((int)m0 + i >= mend) break;
+        uint32_t res[4];
+#pragma unroll
+        for (int c = 0; c < 8; c += 2) {
+            float v[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float qf = __fsub_rn(__int_as_float(0x4B000000 | (int)((wd[i] >> (4 * (c + e))) & 15u)), 8388608.0f);
+                v[e] = __fmul_rn(__fsub_rn(qf, zf[c + e]), df[c + e]);
+            }
+            const __half2 h2 = __floats2half2_rn(v[0], v[1]);
+            memcpy(&res[c / 2], &h2, 4);
+        }
+        __stcs(reinterpret_cast<uint4 *>(out) + (m0 + i) * wpg + j, make_uint4(res[0], res[1], res[2], res[3]));
+    }
+}
+
 template <int NB>
 cudaError_t launch_dequant(const uint8_t *pk, const __half *sc, const __half *ze, int64_t N, int g,
                     int64_t G, int axis, int64_t pb, __half *out, cudaStream_t st) {
@@ -254,6 +304,13 @@ cudaError_t launch_dequant(const uint8_t *pk, const __half *sc, const __half *ze
     }
     if (axis == 1)
         return launch_pdl(hqq_dequant_kernel<NB, 1>, blocks, kDqThreads, 0, st, pw, sc, ze, N, g, G, pb, -1, false, out);
+    // axis 0, 4-bit, whole 8-group words in every stripe (G % 8 == 0 and N = g G), aligned
+    if (NB == 4 && G % 8 == 0 && N == (int64_t)g * G && vec_meta && ((uintptr_t)pk & 15) == 0 &&
+        ((uintptr_t)out & 15) == 0) {
+        const int64_t threads = (G / 8) * ((g + kDqA0M - 1) / kDqA0M);
+        return launch_pdl(hqq_dequant_a0_kernel, (unsigned)((threads + kDqThreads - 1) / kDqThreads), kDqThreads, 0, st,
+                          pw, sc, ze, G, g, out);
+    }
     return launch_pdl(hqq_dequant_kernel<NB, 2>, blocks, kDqThreads, 0, st, pw, sc, ze, N, g, G, pb, -1, vec_meta, out);
 }
 

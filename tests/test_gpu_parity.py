@@ -156,7 +156,10 @@ def test_full_size_config(case, pool):
                                           ((41, 40), 8, 0),
                                           # 3-bit, groups of 40 and more: four words per thread,
                                           # groups that straddle them, a ragged last unit
-                                          ((33, 200), 40, 1), ((7, 130), 65, 1), ((96, 160), 96, 1)])
+                                          ((33, 200), 40, 1), ((7, 130), 65, 1), ((96, 160), 96, 1),
+                                          # axis 0, 4-bit metadata reuse: g = 24 rows (a short
+                                          # last run of words per thread), 128 groups
+                                          ((24, 128), 24, 0)])
 def test_dequant_random_codes(nbits, shape, g, axis):
     from free_weight_quantization_b200 import hqq
     rows, cols = shape

@@ -675,6 +675,59 @@ __global__ void __launch_bounds__(256, 2) hqq_gemv3_kernel(const uint8_t *__rest
     }
 }
 
+// Axis 0, 4-bit, g dividing rows, cols a multiple of 32: element (r, c) is in group
+// (r mod R) cols + c with R = rows / g, so a row's groups are cols consecutive ones and every
+// code has its own scale and zero (read through L2: the R rows of metadata are shared by the g
+// rows of each stripe).  One warp per row; lane l takes pieces of 32 codes l, l + 32, ..., with
+// the piece's 32 zeros, scales and x values as 16-byte loads; pairs are dequantized in packed
+// binary32 exactly as dequantize does and multiplied with x in packed FMAs.
+template <int NB>
+__global__ void __launch_bounds__(256, 3) hqq_gemv_a0_kernel(const uint8_t *__restrict__ packed,
+                                                             const __half *__restrict__ scale,
+                                                             const __half *__restrict__ zero,
+                                                             int64_t rows, int ppr, int R,
+                                                             const __half *__restrict__ x,
+                                                             float *__restrict__ y) {
+    static_assert(NB == 4, "4-bit codes");
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    wait_prerequisite();  // codes and x may come from the kernel launched just before
+    allow_dependents();
+    if (row >= rows) return;  // whole warps
+    const int64_t cols = (int64_t)ppr * 32;
+    const uint8_t *crow = packed + row * cols / 2;
+    const __half *zrow = zero + (row % R) * cols, *srow = scale + (row % R) * cols;
+    const float2 nm = make_float2(-8388608.0f, -8388608.0f);
+    float2 acc = make_float2(0.0f, 0.0f);
+    for (int p = lane; p < ppr; p += 32) {
+        const uint4 cv = __ldcs(reinterpret_cast<const uint4 *>(crow + (int64_t)p * 16));
+        const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {  // word wi: codes 8 wi .. 8 wi + 7 of the piece
+            const uint4 zv = __ldg(reinterpret_cast<const uint4 *>(zrow + (int64_t)p * 32) + wi);
+            const uint4 sv = __ldg(reinterpret_cast<const uint4 *>(srow + (int64_t)p * 32) + wi);
+            const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(x + (int64_t)p * 32) + wi);
+            const uint32_t zs[4] = {zv.x, zv.y, zv.z, zv.w}, ss[4] = {sv.x, sv.y, sv.z, sv.w};
+            const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w};
+            const uint32_t ev = cw[wi] & 0x0F0F0F0Fu, od = (cw[wi] >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {  // codes 2i, 2i + 1 of the word
+                const float2 q = make_float2(__uint_as_float(__byte_perm(ev, 0x4B000000u, 0x7540u + i)),
+                                             __uint_as_float(__byte_perm(od, 0x4B000000u, 0x7540u + i)));
+                const float2 zf = __half22float2(*reinterpret_cast<const __half2 *>(&zs[i]));
+                const float2 df = __half22float2(*reinterpret_cast<const __half2 *>(&ss[i]));
+                const float2 v = __fmul2_rn(__fadd2_rn(__fadd2_rn(q, nm), make_float2(-zf.x, -zf.y)), df);
+                const float2 xf = __half22float2(*reinterpret_cast<const __half2 *>(&xs[i]));
+                acc = __ffma2_rn(__half22float2(__floats2half2_rn(v.x, v.y)), xf, acc);
+            }
+        }
+    }
+    float s = __fadd_rn(acc.x, acc.y);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s = __fadd_rn(s, __shfl_xor_sync(kFull, s, off));
+    if (lane == 0) y[row] = s;
+}
+
 // Any other layout: one warp per output row, each lane takes columns lane, lane + 32, ...
 // and reads its codes one at a time (flat row-major code order, groups by axis).
 template <int NB>
@@ -753,6 +806,13 @@ cudaError_t launch_gemv_nb(const uint8_t *pk, const __half *sc, const __half *ze
             return launch_pdl(hqq_gemv_kernel<NB>, blocks, 256, 0, st, (const uint32_t *)pk, sc, ze,
                               rows, (int)wpr, (int)(cols / g), shift, wpg, x, y);
         }
+    }
+    if constexpr (NB == 4) {  // axis 0 with whole stripes of rows: per-code metadata by row
+        if (axis == 0 && rows % g == 0 && cols % 32 == 0 && cols / 32 < ((int64_t)1 << 30) &&
+            rows / g < ((int64_t)1 << 30) &&
+            ((((uintptr_t)x | (uintptr_t)pk | (uintptr_t)sc | (uintptr_t)ze) & 15) == 0))
+            return launch_pdl(hqq_gemv_a0_kernel<NB>, blocks, 256, 0, st, pk, sc, ze, rows, (int)(cols / 32),
+                              (int)(rows / g), x, y);
     }
     return launch_pdl(hqq_gemv_any_kernel<NB>, blocks, 256, 0, st, pk, sc, ze, rows, cols, g, G,
                       axis, x, y);

@@ -52,7 +52,9 @@ LAYOUTS = [(4, 64, 1, 96, 512), (2, 16, 1, 64, 256), (4, 128, 1, 33, 1024), (2, 
            (4, 64, 1, 40, 96), (2, 32, 1, 30, 48),
            # 16 MiB of codes and more: the bulk-copy kernel; 8195 rows end in a 3-row stage
            # whose 195 metadata halves are not whole 16-byte units (65 groups per row)
-           (4, 64, 1, 8195, 4160), (2, 64, 1, 8192, 8192)]
+           (4, 64, 1, 8195, 4160), (2, 64, 1, 8192, 8192),
+           # axis 0, 4 bit, g dividing rows: per-code metadata by row (stripes of R = rows / g)
+           (4, 32, 0, 96, 64), (4, 8, 0, 40, 320)]
 
 
 @pytest.mark.parametrize("nbits,g,axis,rows,cols", LAYOUTS, ids=lambda v: str(v))
@@ -102,7 +104,7 @@ def test_gemv_unaligned_x_takes_the_generic_path(hqq):
     _check(y, ref, mag, cols, "unaligned x")
 
 
-@pytest.mark.parametrize("case", [wl.ATTN, wl.MLP_B2], ids=lambda c: c.name)
+@pytest.mark.parametrize("case", [wl.ATTN, wl.MLP_B2, wl.ATTN_AX0], ids=lambda c: c.name)
 def test_gemv_on_quantized_workload(hqq, case):
     # the full-size workload quantized on the GPU, then the fused product against the oracle's
     # product of the same packed codes and metadata

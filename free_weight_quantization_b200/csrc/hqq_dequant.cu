@@ -728,6 +728,86 @@ __global__ void __launch_bounds__(256, 3) hqq_gemv_a0_kernel(const uint8_t *__re
     if (lane == 0) y[row] = s;
 }
 
+// 3-bit codes, axis 1, g >= 10, cols even: words of 10 codes may straddle rows (cols need not be
+// a multiple of 10).  One warp per row; the CTA first copies x into shared memory, so that the
+// 10 x values of a word, at any offset, are five 4-byte shared loads (cols is even, so code
+// pairs (2i, 2i + 1) of a word sit at even columns).  A word lies in at most two groups; codes
+// outside the row contribute nothing.  Values as dequantize computes them, products and sums in
+// binary32.
+template <int NB>
+__global__ void __launch_bounds__(256) hqq_gemv_b3_kernel(const uint32_t *__restrict__ packed,
+                                                          const __half *__restrict__ scale,
+                                                          const __half *__restrict__ zero,
+                                                          int64_t rows, int64_t cols, int g, int64_t G,
+                                                          const __half *__restrict__ x,
+                                                          float *__restrict__ y) {
+    static_assert(NB == 3, "3-bit codes");
+    extern __shared__ __align__(16) unsigned char smem[];
+    __half *xs = reinterpret_cast<__half *>(smem);
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    wait_prerequisite();  // codes and x may come from the kernel launched just before
+    allow_dependents();
+    for (int64_t i = threadIdx.x; i < cols / 2; i += blockDim.x)
+        reinterpret_cast<uint32_t *>(xs)[i] = __ldg(reinterpret_cast<const uint32_t *>(x) + i);
+    __syncthreads();
+    if (row >= rows) return;  // whole warps
+    const int64_t nb = row * cols, ne = nb + cols;  // the row's flat code range
+    const int64_t w0 = nb / 10, w1 = (ne - 1) / 10;
+    constexpr int U = 4;  // words per lane loaded before any is used
+    float acc = 0.0f;
+    for (int64_t wb = w0 + lane; wb <= w1; wb += 32 * U) {
+        uint32_t wd[U];
+        float za[U], da[U], zb[U], db[U];
+        int cb[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t w = wb + 32 * u;
+            wd[u] = 0u;
+            za[u] = da[u] = zb[u] = db[u] = 0.0f;
+            cb[u] = 10;
+            if (w <= w1) {
+                wd[u] = __ldcs(packed + w);
+                const int64_t n0 = 10 * w, k0 = n0 / g;
+                cb[u] = (int)(g - (n0 - k0 * g));  // codes j < cb belong to group k0
+                const int64_t k1 = cb[u] < 10 && k0 + 1 < G ? k0 + 1 : k0;  // past the last group: padding
+                za[u] = __half2float(__ldg(zero + k0));
+                da[u] = __half2float(__ldg(scale + k0));
+                zb[u] = __half2float(__ldg(zero + k1));
+                db[u] = __half2float(__ldg(scale + k1));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t w = wb + 32 * u;
+            if (w > w1) break;
+            const int64_t n0 = 10 * w;
+            const bool whole = n0 >= nb && n0 + 10 <= ne;
+#pragma unroll
+            for (int j = 0; j < 10; j += 2) {
+                float v[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int jj = j + e;
+                    const float qf = __fsub_rn(__int_as_float(0x4B000000 | (int)((wd[u] >> (3 * jj)) & 7u)), 8388608.0f);
+                    const bool first = jj < cb[u];
+                    v[e] = __fmul_rn(__fsub_rn(qf, first ? za[u] : zb[u]), first ? da[u] : db[u]);
+                }
+                const float2 wh = __half22float2(__floats2half2_rn(v[0], v[1]));
+                const int64_t c = n0 + j - nb;  // column of code j (even)
+                if (whole || (c >= 0 && c + 1 < cols)) {  // both codes in the row
+                    const float2 xf = __half22float2(*reinterpret_cast<const __half2 *>(xs + c));
+                    acc = __fmaf_rn(wh.x, xf.x, acc);
+                    acc = __fmaf_rn(wh.y, xf.y, acc);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(kFull, acc, off));
+    if (lane == 0) y[row] = acc;
+}
+
 // Any other layout: one warp per output row, each lane takes columns lane, lane + 32, ...
 // and reads its codes one at a time (flat row-major code order, groups by axis).
 template <int NB>
@@ -806,6 +886,11 @@ cudaError_t launch_gemv_nb(const uint8_t *pk, const __half *sc, const __half *ze
             return launch_pdl(hqq_gemv_kernel<NB>, blocks, 256, 0, st, (const uint32_t *)pk, sc, ze,
                               rows, (int)wpr, (int)(cols / g), shift, wpg, x, y);
         }
+    }
+    if constexpr (NB == 3) {  // axis 1, x staged in shared memory (at most 48 KB of it)
+        if (axis == 1 && g >= 10 && cols % 2 == 0 && cols * 2 <= 48 * 1024 && ((uintptr_t)x & 3) == 0)
+            return launch_pdl(hqq_gemv_b3_kernel<NB>, blocks, 256, (int)(cols * 2), st,
+                              reinterpret_cast<const uint32_t *>(pk), sc, ze, rows, cols, (int)g, G, x, y);
     }
     if constexpr (NB == 4) {  // axis 0 with whole stripes of rows: per-code metadata by row
         if (axis == 0 && rows % g == 0 && cols % 32 == 0 && cols / 32 < ((int64_t)1 << 30) &&

@@ -54,7 +54,10 @@ LAYOUTS = [(4, 64, 1, 96, 512), (2, 16, 1, 64, 256), (4, 128, 1, 33, 1024), (2, 
            # whose 195 metadata halves are not whole 16-byte units (65 groups per row)
            (4, 64, 1, 8195, 4160), (2, 64, 1, 8192, 8192),
            # axis 0, 4 bit, g dividing rows: per-code metadata by row (stripes of R = rows / g)
-           (4, 32, 0, 96, 64), (4, 8, 0, 40, 320)]
+           (4, 32, 0, 96, 64), (4, 8, 0, 40, 320),
+           # 3 bit, axis 1: rows that start and end inside a 10-code word, groups not a
+           # multiple of 10
+           (3, 64, 1, 16, 1004), (3, 12, 1, 7, 96)]
 
 
 @pytest.mark.parametrize("nbits,g,axis,rows,cols", LAYOUTS, ids=lambda v: str(v))
@@ -104,7 +107,7 @@ def test_gemv_unaligned_x_takes_the_generic_path(hqq):
     _check(y, ref, mag, cols, "unaligned x")
 
 
-@pytest.mark.parametrize("case", [wl.ATTN, wl.MLP_B2, wl.ATTN_AX0], ids=lambda c: c.name)
+@pytest.mark.parametrize("case", [wl.ATTN, wl.MLP_B2, wl.MLP_B3, wl.ATTN_AX0], ids=lambda c: c.name)
 def test_gemv_on_quantized_workload(hqq, case):
     # the full-size workload quantized on the GPU, then the fused product against the oracle's
     # product of the same packed codes and metadata

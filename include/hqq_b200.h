@@ -145,9 +145,17 @@ int hqq_dequantize(const void *packed, const void *scale, const void *zero, int6
  *   x       [cols] fp16, 2-byte aligned. 16-byte alignment enables the fast path.
  *   y       [rows] binary32, 4-byte aligned (output)
  *   stream  cudaStream_t, or NULL for the default stream
- * Every layout is accepted. The fast path (one warp per output row) needs axis 1, 2- or 4-bit
- * codes, cols and group_size multiples of the codes per 32-bit word (8 at 4 bit, 16 at 2 bit),
- * and group_size dividing cols. Other layouts read their codes one at a time.
+ * Every layout is accepted.  Fast paths (x 16-byte aligned):
+ *   - axis 1, 2- or 4-bit codes, group_size a multiple of 32 dividing cols: one warp per row,
+ *     32-code pieces (from 16 MiB of codes on, with scale and zero 16-byte aligned, rows move
+ *     in bulk copies through shared memory);
+ *   - axis 1, 2- or 4-bit codes, cols and group_size multiples of the codes per 32-bit word (8
+ *     at 4 bit, 16 at 2 bit), group_size dividing cols: one warp per row, one word per load;
+ *   - axis 0, 4-bit codes, group_size dividing rows, cols a multiple of 32, scale and zero
+ *     16-byte aligned: one warp per row with per-code metadata;
+ *   - axis 1, 3-bit codes, group_size >= 10, cols even and at most 24576, x 4-byte aligned
+ *     suffices: x staged in shared memory.
+ * Other layouts read their codes one at a time.
  * Returns HQQ_OK, HQQ_ERR_ARG (shape or null pointer), HQQ_ERR_ALIGN, or HQQ_ERR_CUDA.
  */
 int hqq_gemv(const void *packed, const void *scale, const void *zero, int64_t rows, int64_t cols,

@@ -12,6 +12,10 @@ namespace {
 //   MODE 0: axis 1, group_size a multiple of the codes per word: one group per word
 //   MODE 1: axis 1, any group size
 //   MODE 2: axis 0 (element n belongs to group n % G)
+//   MODE 3: axis 1, group_size at least the codes per word: a word spans two groups at most
+// Two more kernels below take layouts these serve less well: 3-bit codes four words per thread
+// (16-byte stores), and axis-0 4-bit codes with each word's metadata loaded once per column.
+// The forward products follow them.
 // ------------------------------------------------------------------------------------------
 constexpr int kDqU = 4;
 constexpr int kDqThreads = 256;

@@ -69,6 +69,14 @@ def test_workspace_bytes(L):
     assert ws(16, 16, 4, 16, 1, 65) == 0       # iters beyond the library limit
     # axis=0 whose packed words do not line up with tiles needs byte staging of all codes
     assert ws(8, 6, 4, 2, 0, 20) >= 48
+    # a small stream-engine tensor (at most 16384 groups) also keeps each group's zero after
+    # every update, G x iters binary32; a large one, the tile engine and iters = 0 do not
+    small = ws(256, 512, 4, 64, 1, 20)
+    assert small >= 2048 * 20 * 4
+    assert ws(256, 512, 4, 64, 1, 10) <= small - 2048 * 10 * 4
+    assert ws(256, 512, 3, 64, 1, 20) < 2048 * 20 * 4      # 3 bit: the tile engine
+    assert ws(256, 512, 4, 64, 1, 0) < 2048 * 4
+    assert ws(4096, 4096, 4, 64, 1, 20) < G + 65536          # 262144 groups: none
 
 
 FAKE = 0x10000  # never dereferenced: every call below fails its host-side checks first

@@ -144,12 +144,13 @@ def hqq_quantize(W: torch.Tensor, nbits: int = 4, group_size: int = 64, axis: in
         workspace = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
     opt = HqqOpt(iters, lp_norm, beta, kappa, eps_tiny, scale_max)
     st = stream if stream is not None else torch.cuda.current_stream(dev)
-    rc = lib().hqq_quantize(_ptr(W), rows, cols, nbits, group_size, axis, ctypes.byref(opt),
-                            _ptr(out.packed), _ptr(out.scale), _ptr(out.zero), _ptr(out.iters_run),
-                            _ptr(out.s), _ptr(out.z), _ptr(out.err_trace), _ptr(out.rounds),
-                            _ptr(workspace),
-                            workspace.numel() * workspace.element_size(),
-                            ctypes.c_void_p(st.cuda_stream))
+    with torch.cuda.device(dev):  # launches go to the current device: W's
+        rc = lib().hqq_quantize(_ptr(W), rows, cols, nbits, group_size, axis, ctypes.byref(opt),
+                                _ptr(out.packed), _ptr(out.scale), _ptr(out.zero), _ptr(out.iters_run),
+                                _ptr(out.s), _ptr(out.z), _ptr(out.err_trace), _ptr(out.rounds),
+                                _ptr(workspace),
+                                workspace.numel() * workspace.element_size(),
+                                ctypes.c_void_p(st.cuda_stream))
     _check(rc, "hqq_quantize")
     return out
 
@@ -195,8 +196,9 @@ def hqq_dequantize(q: Quantized, out: torch.Tensor | None = None,
     if out is None:
         out = torch.empty(q.rows, q.cols, dtype=torch.float16, device=q.packed.device)
     st = stream if stream is not None else torch.cuda.current_stream(q.packed.device)
-    rc = lib().hqq_dequantize(_ptr(q.packed), _ptr(q.scale), _ptr(q.zero), q.rows, q.cols, q.nbits,
-                              q.group_size, q.axis, _ptr(out), ctypes.c_void_p(st.cuda_stream))
+    with torch.cuda.device(q.packed.device):
+        rc = lib().hqq_dequantize(_ptr(q.packed), _ptr(q.scale), _ptr(q.zero), q.rows, q.cols, q.nbits,
+                                  q.group_size, q.axis, _ptr(out), ctypes.c_void_p(st.cuda_stream))
     _check(rc, "hqq_dequantize")
     return out
 
@@ -210,8 +212,9 @@ def hqq_gemv(q: Quantized, x: torch.Tensor, out: torch.Tensor | None = None,
     if out is None:
         out = torch.empty(q.rows, dtype=torch.float32, device=q.packed.device)
     st = stream if stream is not None else torch.cuda.current_stream(q.packed.device)
-    rc = lib().hqq_gemv(_ptr(q.packed), _ptr(q.scale), _ptr(q.zero), q.rows, q.cols, q.nbits,
-                        q.group_size, q.axis, _ptr(x), _ptr(out), ctypes.c_void_p(st.cuda_stream))
+    with torch.cuda.device(q.packed.device):
+        rc = lib().hqq_gemv(_ptr(q.packed), _ptr(q.scale), _ptr(q.zero), q.rows, q.cols, q.nbits,
+                            q.group_size, q.axis, _ptr(x), _ptr(out), ctypes.c_void_p(st.cuda_stream))
     _check(rc, "hqq_gemv")
     return out
 
@@ -226,8 +229,9 @@ def hqq_gemm(q: Quantized, X: torch.Tensor, out: torch.Tensor | None = None,
     if out is None:
         out = torch.empty(batch, q.rows, dtype=torch.float32, device=q.packed.device)
     st = stream if stream is not None else torch.cuda.current_stream(q.packed.device)
-    rc = lib().hqq_gemm(_ptr(q.packed), _ptr(q.scale), _ptr(q.zero), q.rows, q.cols, q.nbits,
-                        q.group_size, q.axis, _ptr(X), batch, _ptr(out), ctypes.c_void_p(st.cuda_stream))
+    with torch.cuda.device(q.packed.device):
+        rc = lib().hqq_gemm(_ptr(q.packed), _ptr(q.scale), _ptr(q.zero), q.rows, q.cols, q.nbits,
+                            q.group_size, q.axis, _ptr(X), batch, _ptr(out), ctypes.c_void_p(st.cuda_stream))
     _check(rc, "hqq_gemm")
     return out
 
